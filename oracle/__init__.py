@@ -1,0 +1,187 @@
+"""fp64 CPU oracle for the indexed sparse attention (DSA) hot path.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg import this package. The product path (the CUDA
+library and its Python binding) never imports, loads or calls it, and the two
+share no code: the only common module is the seeded input generator, which
+holds none of the method's arithmetic.
+
+The arithmetic lives in ``dsa_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module builds it with gcc on first use and wraps it with numpy.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsa_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+
+
+def build(force: bool = False) -> str:
+    """Compile dsa_oracle.c into liboracle.so next to it (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", _SRC, "-o", tmp, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            lib.oracle_e4m3_decode.restype = ctypes.c_double
+            lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+            lib.oracle_e4m3_encode_satfinite.restype = ctypes.c_uint8
+            lib.oracle_e4m3_encode_satfinite.argtypes = [ctypes.c_float]
+            lib.oracle_quantize_keys.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _u8p, _f32p]
+            lib.oracle_dequantize_keys.argtypes = [_u8p, _f32p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _f32p]
+            lib.oracle_indexer_scores.argtypes = [
+                ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, _i32p, ctypes.c_int32, ctypes.c_int32,
+                _f32p, _f32p, ctypes.c_int32, _f32p, _u8p, _f32p, ctypes.c_int32,
+                ctypes.c_int32, _i32p, _f64p, ctypes.c_int64]
+            lib.oracle_topk.argtypes = [ctypes.c_int32, _f64p, ctypes.c_int64, _i32p, ctypes.c_int32, _i32p]
+            lib.oracle_sparse_mla.argtypes = [
+                ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                ctypes.c_double, _f32p, _f32p, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32, _f64p, _f64p]
+            lib.oracle_num_threads.restype = ctypes.c_int32
+            lib.oracle_set_num_threads.argtypes = [ctypes.c_int32]
+            _lib = lib
+    return _lib
+
+
+def _p(a, t):
+    return a.ctypes.data_as(t)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().oracle_set_num_threads(int(n))
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Decode E4M3 codes (uint8 array) to fp64 per the OCP FP8 definition."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_decode(int(v)) for v in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Round fp32 values to E4M3 codes (nearest-even, saturating to +-448)."""
+    lib = _load()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([lib.oracle_e4m3_encode_satfinite(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def quantize_keys(k: np.ndarray, group: int):
+    """Per-group FP8 cache write of keys [..., dim] -> (codes uint8, scales fp32)."""
+    k = _c(k, np.float32)
+    dim = k.shape[-1]
+    n = k.size // dim
+    codes = np.empty(k.shape, np.uint8)
+    scales = np.empty(k.shape[:-1] + (dim // group,), np.float32)
+    _load().oracle_quantize_keys(_p(k, _f32p), n, dim, group, _p(codes, _u8p), _p(scales, _f32p))
+    return codes, scales
+
+
+def dequantize_keys(codes: np.ndarray, scales: np.ndarray, group: int) -> np.ndarray:
+    """fl32(decode(code) * scale) per element."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.float32)
+    dim = codes.shape[-1]
+    n = codes.size // dim
+    out = np.empty(codes.shape, np.float32)
+    _load().oracle_dequantize_keys(_p(codes, _u8p), _p(scales, _f32p), n, dim, group, _p(out, _f32p))
+    return out
+
+
+def indexer_scores(wl, rows=None, *, k_codes=None, k_scales=None) -> np.ndarray:
+    """Oracle scores [len(rows), Lmax] (fp64; -inf where masked) for workload ``wl``.
+
+    FP8 keys are used when ``k_codes``/``k_scales`` are given (dequantised in
+    fp64 inside the oracle); otherwise the bf16 keys ``wl.k_idx``."""
+    lib = _load()
+    rows = np.arange(wl.T, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    out = np.empty((len(rows), wl.Lmax), np.float64)
+    cu_q, q_pos, lens = _c(wl.cu_q, np.int32), _c(wl.q_pos, np.int32), _c(wl.seq_lens, np.int32)
+    q_idx, w = _c(wl.q_idx, np.float32), _c(wl.w, np.float32)
+    if k_codes is not None:
+        k8, ks = _c(k_codes, np.uint8), _c(k_scales, np.float32)
+        kf = np.zeros(1, np.float32)
+        is8 = 1
+        group = wl.dI // ks.shape[-1]
+    else:
+        kf = _c(wl.k_idx, np.float32)
+        k8, ks = np.zeros(1, np.uint8), np.zeros(1, np.float32)
+        is8 = 0
+        group = wl.dI
+    lib.oracle_indexer_scores(wl.B, wl.Lmax, _p(cu_q, _i32p), _p(q_pos, _i32p), _p(lens, _i32p),
+                              wl.HI, wl.dI, _p(q_idx, _f32p), _p(w, _f32p), is8, _p(kf, _f32p),
+                              _p(k8, _u8p), _p(ks, _f32p), group, len(rows), _p(rows, _i32p),
+                              _p(out, _f64p), wl.Lmax)
+    return out
+
+
+def topk(scores: np.ndarray, n_valid, K: int) -> np.ndarray:
+    """Top-K positions per row (ties: higher score, then lower position);
+    ascending by position, padded with -1."""
+    s = _c(scores, np.float64)
+    nv = _c(n_valid, np.int32)
+    out = np.empty((s.shape[0], K), np.int32)
+    _load().oracle_topk(s.shape[0], _p(s, _f64p), s.shape[1], _p(nv, _i32p), K, _p(out, _i32p))
+    return out
+
+
+def sparse_mla(wl, idx: np.ndarray, rows=None):
+    """Attention over the selected rows: returns (out [n,H,dc] fp64, lse [n,H] fp64)."""
+    lib = _load()
+    rows = np.arange(wl.T, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    idx = _c(idx, np.int32)
+    K = idx.shape[1]
+    out = np.empty((len(rows), wl.H, wl.dc), np.float64)
+    lse = np.empty((len(rows), wl.H), np.float64)
+    cu_q, lens = _c(wl.cu_q, np.int32), _c(wl.seq_lens, np.int32)
+    q, kv = _c(wl.q, np.float32), _c(wl.kv, np.float32)
+    lib.oracle_sparse_mla(wl.B, wl.Lmax, _p(cu_q, _i32p), _p(lens, _i32p), wl.H, wl.D, wl.dc,
+                          float(wl.softmax_scale), _p(q, _f32p), _p(kv, _f32p), len(rows),
+                          _p(rows, _i32p), _p(idx, _i32p), K, _p(out, _f64p), _p(lse, _f64p))
+    return out, lse
+
+
+def dsa(wl, rows=None, *, k_codes=None, k_scales=None, rank_in_fp32: bool = False):
+    """The whole hot path for the rows ``rows``: (scores, idx, out, lse).
+
+    ``rank_in_fp32`` ranks the fp64 scores after one rounding to fp32, the
+    precision in which the kernel takes the Top-K decision (used where the
+    scores are exact integers times one fp32 scale)."""
+    rows = np.arange(wl.T, dtype=np.int32) if rows is None else np.asarray(rows, np.int32)
+    sc = indexer_scores(wl, rows, k_codes=k_codes, k_scales=k_scales)
+    rank = sc.astype(np.float32).astype(np.float64) if rank_in_fp32 else sc
+    nv = wl.n_valid()[rows]
+    idx = topk(rank, nv, wl.K)
+    out, lse = sparse_mla(wl, idx, rows)
+    return sc, idx, out, lse
