@@ -1,0 +1,213 @@
+/*
+ * dsa.h -- C ABI of libdsa.so: the indexed sparse attention (DSA) hot path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The path (section 1 of "Day-0 Inference Optimization for a New Sparse
+ * Attention Architecture"; section 3 of "Optimizing Inference for New Model
+ * Architectures: Co-Designing Sparse Attention, State Recurrence, and
+ * Long-Sequence Partitioning"):
+ *   1. Lightning Indexer: relevance scoring of each query token against every
+ *      causal history position, weighted over indexer heads,
+ *        I[t,s] = sum_j w[t,j] * max(0, q_I[t,j,:] . k_I[s,:]),  s <= pos(t);
+ *   2. Top-K: the K highest-scoring positions per query row (ties: higher
+ *      score, then lower position);
+ *   3. Sparse Flash Attention over multi-head latent attention (MLA) rows:
+ *      every query head attends only over the selected latent KV rows; a row
+ *      has d_latent + d_rope dims, the value is its first d_latent dims.
+ * The "pseudocode: fused execution of the sparse attention path" of
+ * "Inference Adaptation and Performance Optimization for New Large Language
+ * Model Architectures" (section 6) splits the path as
+ *   indices = lightning_indexer(query, key_cache)
+ *   output  = sparse_flash_attention(query, indices, key_cache, value_cache)
+ * which the calls below follow: dsa_indexer_scores + dsa_topk form the
+ * indexer, dsa_sparse_mla_attn the attention, dsa_fused_decode the whole
+ * chain. The index-key cache can be BF16 or FP8 E4M3 with a per-group fp32
+ * scale (Tiered Quantization of "Day-0 Inference Adaptation and Performance
+ * Optimization for New-Architecture Large Language Models"); both paths have
+ * the same interface ("the quantized path maintains the same interface
+ * semantics as the high-precision path", Layered Quantization of "Inference
+ * Optimization for New Open-Source LLM Architectures ...").
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers unless stated, row-major, owned
+ *    by the caller. The library allocates no device memory, keeps no per-call
+ *    state and never synchronises (except dsa_read_device_status), so every
+ *    call can be enqueued inside CUDA stream capture.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).
+ *  - Argument, shape and alignment errors return a status before anything is
+ *    enqueued; dsa_last_error() then describes the problem.
+ *  - A failed kernel launch returns DSA_ERR_CUDA.
+ *  - Errors found on the device (an index that is neither -1 nor inside
+ *    [0, seq_len), or a bounded wait inside a kernel that gave up) never trap:
+ *    the offending element is skipped and a sticky per-device status word is
+ *    set; read it with dsa_read_device_status().
+ *  - Supported shapes: indexer heads H_I in [1, 64] with H_I * (tokens per
+ *    group) <= 256, indexer dim d_I in {32, 64, 128}; MLA (d_latent, d_rope)
+ *    in {(512, 64), (64, 16)}; MLA heads H in [1, 128] (a multiple of 64 or
+ *    smaller than 64); 1 <= K <= 2048. Others return
+ *    DSA_ERR_UNSUPPORTED_SHAPE.
+ *  - Alignment: every tensor pointer must be 16-byte aligned.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *dsa_stream_t; /* same type as cudaStream_t */
+typedef struct CUevent_st *dsa_event_t;   /* same type as cudaEvent_t */
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARGUMENT = 1,   /* null pointer, negative size, bad enum */
+    DSA_ERR_UNSUPPORTED_SHAPE = 2,  /* outside the supported shapes above */
+    DSA_ERR_WORKSPACE_TOO_SMALL = 3,/* ws_bytes < dsa_workspace_size(...) */
+    DSA_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
+    DSA_ERR_DEVICE_INDEX = 5,       /* device status: an index out of range was skipped */
+    DSA_ERR_DEVICE_TIMEOUT = 6,     /* device status: a bounded wait gave up */
+    DSA_ERR_MISALIGNED = 7          /* a pointer is not 16-byte aligned */
+} dsa_status;
+
+typedef enum { DSA_KEY_BF16 = 0, DSA_KEY_FP8_E4M3 = 1 } dsa_key_dtype;
+
+/* Ops for dsa_workspace_size(). */
+typedef enum {
+    DSA_OP_INDEXER_SCORES = 0,
+    DSA_OP_TOPK = 1,
+    DSA_OP_SPARSE_MLA = 2,
+    DSA_OP_FUSED_DECODE = 3
+} dsa_op;
+
+/* The batch: B sequences, T query tokens packed sequence after sequence.
+ *   cu_q     [B+1] int32 device: tokens of sequence b are [cu_q[b], cu_q[b+1]);
+ *                  cu_q[0] = 0, non-decreasing, cu_q[B] = T.
+ *   q_pos    [T]   int32 device: position of each query token inside its
+ *                  sequence; its causal history is s <= q_pos.
+ *   seq_lens [B]   int32 device: valid cache rows of sequence b (<= max_seq_len).
+ *   max_seq_len    L_max, the row stride of the caches: sequence b's rows are
+ *                  cache[b * L_max + s].
+ *   block_table / page_size: reserved for paged caches; must be NULL / 0.
+ * A query's candidate count is n_valid(t) = min(q_pos[t] + 1, seq_lens[b]). */
+typedef struct {
+    int32_t batch;
+    int32_t num_q;
+    int32_t max_seq_len;
+    const int32_t *cu_q;
+    const int32_t *q_pos;
+    const int32_t *seq_lens;
+    const int32_t *block_table;
+    int32_t page_size;
+} dsa_batch;
+
+/* Lightning Indexer inputs.
+ *   q        bf16 [T, n_heads, head_dim]       indexer queries q_I
+ *   w        fp32 [T, n_heads]                 head weights
+ *   k_cache  [B, L_max, head_dim]              index keys, bf16 or e4m3 codes
+ *   k_scale  fp32 [B, L_max, head_dim/scale_group] per-group scales (FP8 only;
+ *            the key value is decode(code) * scale), NULL for BF16
+ *   scale_group: elements per scale; must equal head_dim for the FP8 indexer. */
+typedef struct {
+    int32_t n_heads;
+    int32_t head_dim;
+    const void *q;
+    const float *w;
+    dsa_key_dtype key_dtype;
+    const void *k_cache;
+    const float *k_scale;
+    int32_t scale_group;
+} dsa_indexer_in;
+
+/* Sparse MLA inputs.
+ *   q   bf16 [T, n_heads, d_latent + d_rope]
+ *   kv  bf16 [B, L_max, d_latent + d_rope]   latent rows; value = first d_latent
+ *   softmax_scale: multiplies q . kv before the softmax. */
+typedef struct {
+    int32_t n_heads;
+    int32_t d_latent;
+    int32_t d_rope;
+    float softmax_scale;
+    const void *q;
+    const void *kv;
+} dsa_mla_in;
+
+/* Lightning Indexer scores (relevance scoring + head-weight weighting +
+ * causal/ragged mask).
+ * scores: fp32 [T, score_ld], score_ld >= max_seq_len. Row t gets
+ *   I[t,s] for s < n_valid(t) and -inf for n_valid(t) <= s < the end of the
+ *   last 128-key tile that holds a valid key; entries beyond are not written.
+ * FP8 keys: I = scale_s * sum_j w_j * max(0, q_j . decode(code_s)), which
+ * equals the score of the dequantised key because scale_s >= 0.
+ * ws: workspace of dsa_workspace_size(DSA_OP_INDEXER_SCORES, ...) bytes (may
+ * be NULL when that size is 0). */
+dsa_status dsa_indexer_scores(const dsa_batch *batch, const dsa_indexer_in *in, float *scores,
+                              int64_t score_ld, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Per-row Top-K of the indexer scores.
+ * scores: fp32 [T, score_ld]; only columns [0, n_valid(t)) are read.
+ * idx: int32 [T, k]: the min(k, n_valid(t)) best positions of row t under the
+ *   order (score desc, position asc) with -0 == +0, written in ascending
+ *   position order and padded with -1. Bit-identical for identical scores. */
+dsa_status dsa_topk(const dsa_batch *batch, const float *scores, int64_t score_ld, int32_t k,
+                    int32_t *idx, void *ws, size_t ws_bytes, dsa_stream_t stream);
+
+/* Sparse MLA attention over the selected rows.
+ * idx: int32 [T, k]; -1 entries are skipped; entries outside [0, seq_len) are
+ *   skipped and set DSA_ERR_DEVICE_INDEX in the device status word.
+ * out: bf16 [T, n_heads, d_latent]:  sum_i softmax_i(scale * q.kv_i) * kv_i[0:d_latent]
+ * lse: fp32 [T, n_heads] natural-log sum-exp of the scaled logits, or NULL.
+ * A row with no valid index gets out = 0 and lse = -inf.
+ * ws: dsa_workspace_size(DSA_OP_SPARSE_MLA, ...) bytes (split-K partials). */
+dsa_status dsa_sparse_mla_attn(const dsa_batch *batch, const dsa_mla_in *in, const int32_t *idx,
+                               int32_t k, void *out, float *lse, void *ws, size_t ws_bytes,
+                               dsa_stream_t stream);
+
+/* The whole decode chain: indexer scores -> Top-K -> sparse MLA, enqueued
+ * back to back on `stream` with intermediates in the workspace.
+ * idx_out: if non-NULL, int32 [T, k] receives the selected indices.
+ * stage_events: NULL, or 4 caller-created events recorded before the indexer,
+ *   before the Top-K, before the attention and after the attention (timing).
+ * ws: dsa_workspace_size(DSA_OP_FUSED_DECODE, ...) bytes. */
+dsa_status dsa_fused_decode(const dsa_batch *batch, const dsa_indexer_in *idx_in,
+                            const dsa_mla_in *mla_in, int32_t k, void *out, float *lse,
+                            int32_t *idx_out, void *ws, size_t ws_bytes,
+                            const dsa_event_t *stage_events, dsa_stream_t stream);
+
+/* Index-key cache write: per-group dynamic FP8 quantisation.
+ * k_bf16: bf16 [n_keys, dim]; for every group of `group` elements
+ *   scale = fl32(max|k| / 448); scale == 0 -> codes 0;
+ *   else code = e4m3 round-to-nearest-even, saturating, of fl32(k / scale).
+ * k8: uint8 [n_keys, dim]; scale: fp32 [n_keys, dim/group].
+ * group in {32, 64, 128}, dim a multiple of group and of 4, dim <= 1024. */
+dsa_status dsa_quantize_index_keys(const void *k_bf16, int64_t n_keys, int32_t dim, int32_t group,
+                                   uint8_t *k8, float *scale, dsa_stream_t stream);
+
+/* Dequantisation: out = fl32(decode(code) * scale), fp32 [n_keys, dim]. */
+dsa_status dsa_dequantize_index_keys(const uint8_t *k8, const float *scale, int64_t n_keys,
+                                     int32_t dim, int32_t group, float *out, dsa_stream_t stream);
+
+/* Workspace bytes `op` needs for this batch, k and indexer shape (h_i, d_i);
+ * the MLA shape is fixed by the supported set, the largest is assumed.
+ * Host-only: reads no device memory. */
+size_t dsa_workspace_size(int op, const dsa_batch *batch, int32_t k, int32_t h_i, int32_t d_i);
+
+/* Waits for `stream`, then returns in *code_out the sticky device status
+ * (DSA_OK or a DSA_ERR_DEVICE_* code) of the current device and clears it. */
+dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t *code_out);
+
+/* Text for a status code (static storage). */
+const char *dsa_status_string(dsa_status s);
+
+/* Detail of the last non-OK return on the calling thread (static per thread). */
+const char *dsa_last_error(void);
+
+/* Library version string. */
+const char *dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSA_H_ */

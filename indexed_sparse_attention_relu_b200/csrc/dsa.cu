@@ -1,0 +1,474 @@
+// dsa.cu -- host side of libdsa.so: argument validation, workspace planning,
+// tensor-map encoding and kernel launches for the DSA hot path (the C ABI of
+// include/dsa.h). All kernels live in this translation unit so they share the
+// device status word.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "dsa_common.cuh"
+#include "indexer.cuh"
+#include "quant.cuh"
+#include "sparse_mla.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using namespace dsa;
+
+thread_local char g_last_error[512] = "";
+
+dsa_status fail(dsa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+dsa_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 2-D map over the index-key cache: x = element within a key, y = key row.
+dsa_status make_key_map(CUtensorMap* map, const void* base, int64_t rows, int din, bool fp8) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(din), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(din) * (fp8 ? 1u : 2u)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r;
+  if (fp8) {
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(din), 128};
+    r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint32_t box[2] = {64, 128};  // one 128-byte swizzle atom column of 128 keys
+    r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- validation
+dsa_status check_batch(const dsa_batch* bt) {
+  if (!bt) return fail(DSA_ERR_INVALID_ARGUMENT, "batch is NULL");
+  if (bt->batch <= 0 || bt->num_q < 0 || bt->max_seq_len <= 0)
+    return fail(DSA_ERR_INVALID_ARGUMENT, "batch=%d num_q=%d max_seq_len=%d must be positive", bt->batch,
+                bt->num_q, bt->max_seq_len);
+  if (bt->num_q > 0 && (!bt->cu_q || !bt->q_pos || !bt->seq_lens))
+    return fail(DSA_ERR_INVALID_ARGUMENT, "cu_q, q_pos and seq_lens must be non-NULL");
+  if (bt->block_table || bt->page_size)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "paged caches (block_table) are not supported");
+  if (static_cast<int64_t>(bt->batch) * bt->max_seq_len >= (int64_t(1) << 31))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "batch * max_seq_len must be < 2^31");
+  return DSA_OK;
+}
+
+dsa_status check_indexer(const dsa_batch* bt, const dsa_indexer_in* in) {
+  if (!in) return fail(DSA_ERR_INVALID_ARGUMENT, "indexer input is NULL");
+  const bool shape_ok = (in->n_heads == 64 && in->head_dim == 128) || (in->n_heads == 64 && in->head_dim == 32) ||
+                        (in->n_heads == 4 && in->head_dim == 32) || (in->n_heads == 4 && in->head_dim == 128);
+  if (!shape_ok)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "indexer heads/dim %d/%d not in {4,64} x {32,128}", in->n_heads,
+                in->head_dim);
+  if (in->key_dtype != DSA_KEY_BF16 && in->key_dtype != DSA_KEY_FP8_E4M3)
+    return fail(DSA_ERR_INVALID_ARGUMENT, "bad key dtype %d", static_cast<int>(in->key_dtype));
+  if (!in->q || !in->w || !in->k_cache) return fail(DSA_ERR_INVALID_ARGUMENT, "indexer q, w, k_cache must be non-NULL");
+  if (!aligned16(in->q) || !aligned16(in->w) || !aligned16(in->k_cache))
+    return fail(DSA_ERR_MISALIGNED, "indexer q, w, k_cache must be 16-byte aligned");
+  if (in->key_dtype == DSA_KEY_FP8_E4M3) {
+    if (!in->k_scale) return fail(DSA_ERR_INVALID_ARGUMENT, "FP8 keys need k_scale");
+    if (in->scale_group != in->head_dim)
+      return fail(DSA_ERR_UNSUPPORTED_SHAPE, "FP8 indexer needs one scale per key (scale_group == head_dim)");
+  }
+  (void)bt;
+  return DSA_OK;
+}
+
+dsa_status check_mla(const dsa_mla_in* in) {
+  if (!in) return fail(DSA_ERR_INVALID_ARGUMENT, "MLA input is NULL");
+  const bool dims_ok = (in->d_latent == 512 && in->d_rope == 64) || (in->d_latent == 64 && in->d_rope == 16);
+  if (!dims_ok)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "MLA dims (%d,%d) not in {(512,64),(64,16)}", in->d_latent, in->d_rope);
+  if (in->n_heads < 1 || in->n_heads > 128 || (in->n_heads > 64 && in->n_heads % 64 != 0))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "MLA heads %d must be <= 64 or a multiple of 64 up to 128", in->n_heads);
+  if (!in->q || !in->kv) return fail(DSA_ERR_INVALID_ARGUMENT, "MLA q and kv must be non-NULL");
+  if (!aligned16(in->q) || !aligned16(in->kv)) return fail(DSA_ERR_MISALIGNED, "MLA q and kv must be 16-byte aligned");
+  if (!std::isfinite(in->softmax_scale)) return fail(DSA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite");
+  return DSA_OK;
+}
+
+// ---------------------------------------------------------------- planning
+int indexer_group(const dsa_batch* bt) { return bt->num_q > bt->batch ? 4 : 1; }
+
+struct MlaPlan {
+  int splits;
+  int keys_per_split;
+};
+
+MlaPlan mla_plan(int T, int K, int sms) {
+  const int tiles = (K + 63) / 64;
+  int splits = T > 0 ? (sms + T - 1) / T : 1;
+  splits = splits < 1 ? 1 : (splits > tiles ? tiles : splits);
+  const int tps = (tiles + splits - 1) / splits;
+  splits = (tiles + tps - 1) / tps;
+  return MlaPlan{splits, tps * 64};
+}
+
+size_t mla_ws_bytes(int T, int H, int DC, int K, int sms) {
+  const MlaPlan pl = mla_plan(T, K, sms);
+  if (pl.splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(pl.splits) * T * H;
+  return align256(rows * DC * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+// ---------------------------------------------------------------- launches
+template <typename Kern>
+dsa_status set_smem(Kern k, int bytes) {
+  const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+  return DSA_OK;
+}
+
+template <int HI, int DIN, int G, bool FP8>
+dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
+                            cudaStream_t st) {
+  using C = IndexerCfg<HI, DIN, G, FP8>;
+  CUtensorMap map;
+  dsa_status s = make_key_map(&map, in->k_cache, static_cast<int64_t>(bt->batch) * bt->max_seq_len, DIN, FP8);
+  if (s != DSA_OK) return s;
+  auto kern = indexer_scores_kernel<HI, DIN, G, FP8>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
+  const int sms = num_sms();
+  const int64_t groups64 = static_cast<int64_t>((bt->num_q + G - 1) / G) + bt->batch;
+  const int groups = static_cast<int>(groups64 < bt->num_q ? groups64 : bt->num_q);
+  const int max_tiles = (bt->max_seq_len + 127) / 128;
+  int per_group = sms / (groups > 0 ? groups : 1);
+  if (per_group < 1) per_group = 1;
+  int tpc = (max_tiles + per_group - 1) / per_group;
+  if (tpc > 64) tpc = 64;
+  if (tpc < 1) tpc = 1;
+  const int gy = (max_tiles + tpc - 1) / tpc;
+  IndexerParams p;
+  p.cu_q = bt->cu_q;
+  p.q_pos = bt->q_pos;
+  p.seq_lens = bt->seq_lens;
+  p.B = bt->batch;
+  p.L_max = bt->max_seq_len;
+  p.q = static_cast<const __nv_bfloat16*>(in->q);
+  p.w = in->w;
+  p.k_scale = in->k_scale;
+  p.scores = scores;
+  p.ld = ld;
+  p.tiles_per_cta = tpc;
+  kern<<<dim3(groups, gy), C::THREADS, C::SMEM_BYTES, st>>>(map, p);
+  return check_launch("indexer_scores");
+}
+
+template <int HI, int DIN>
+dsa_status launch_indexer_g(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
+                            cudaStream_t st) {
+  const bool fp8 = in->key_dtype == DSA_KEY_FP8_E4M3;
+  if (indexer_group(bt) == 4)
+    return fp8 ? launch_indexer_t<HI, DIN, 4, true>(bt, in, scores, ld, st)
+               : launch_indexer_t<HI, DIN, 4, false>(bt, in, scores, ld, st);
+  return fp8 ? launch_indexer_t<HI, DIN, 1, true>(bt, in, scores, ld, st)
+             : launch_indexer_t<HI, DIN, 1, false>(bt, in, scores, ld, st);
+}
+
+dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
+                          cudaStream_t st) {
+  if (in->n_heads == 64 && in->head_dim == 128) return launch_indexer_g<64, 128>(bt, in, scores, ld, st);
+  if (in->n_heads == 64 && in->head_dim == 32) return launch_indexer_g<64, 32>(bt, in, scores, ld, st);
+  if (in->n_heads == 4 && in->head_dim == 128) return launch_indexer_g<4, 128>(bt, in, scores, ld, st);
+  return launch_indexer_g<4, 32>(bt, in, scores, ld, st);
+}
+
+constexpr int kTopkThreads = 512;
+constexpr int kTopkCacheMax = 49152;  // keys (192 KB)
+
+dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int k, int32_t* idx, cudaStream_t st) {
+  const int cap = bt->max_seq_len < kTopkCacheMax ? bt->max_seq_len : kTopkCacheMax;
+  const int bytes = cap * 4;
+  dsa_status s = set_smem(topk_kernel<kTopkThreads>, bytes);
+  if (s != DSA_OK) return s;
+  TopkParams p;
+  p.scores = scores;
+  p.ld = ld;
+  p.cu_q = bt->cu_q;
+  p.q_pos = bt->q_pos;
+  p.seq_lens = bt->seq_lens;
+  p.B = bt->batch;
+  p.L_max = bt->max_seq_len;
+  p.K = k;
+  p.idx = idx;
+  p.cache_cap = cap;
+  topk_kernel<kTopkThreads><<<bt->num_q, kTopkThreads, bytes, st>>>(p);
+  return check_launch("topk");
+}
+
+template <int D, int DC>
+dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
+                        float* lse, void* ws, cudaStream_t st) {
+  using C = MlaCfg<D, DC>;
+  auto kern = sparse_mla_kernel<D, DC>;
+  dsa_status s = set_smem(kern, C::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  const int T = bt->num_q, H = in->n_heads;
+  const MlaPlan pl = mla_plan(T, k, num_sms());
+  MlaParams p;
+  p.cu_q = bt->cu_q;
+  p.seq_lens = bt->seq_lens;
+  p.B = bt->batch;
+  p.L_max = bt->max_seq_len;
+  p.T = T;
+  p.H = H;
+  p.K = k;
+  p.q = static_cast<const __nv_bfloat16*>(in->q);
+  p.kv = static_cast<const __nv_bfloat16*>(in->kv);
+  p.idx = idx;
+  p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
+  p.keys_per_split = pl.keys_per_split;
+  p.splits = pl.splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  if (pl.splits > 1) {
+    const size_t rows = static_cast<size_t>(pl.splits) * T * H;
+    p.part_o = static_cast<float*>(ws);
+    p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(rows * DC * sizeof(float)));
+  }
+  const int hb = (H + 63) / 64;
+  kern<<<dim3(T, hb, pl.splits), C::THREADS, C::SMEM_BYTES, st>>>(p);
+  if ((s = check_launch("sparse_mla")) != DSA_OK) return s;
+  if (pl.splits > 1) {
+    mla_combine_kernel<<<static_cast<unsigned>(static_cast<int64_t>(T) * H), 128, 0, st>>>(
+        p.part_o, p.part_lse, pl.splits, T, H, DC, p.out, lse);
+    if ((s = check_launch("mla_combine")) != DSA_OK) return s;
+  }
+  return DSA_OK;
+}
+
+dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
+                      void* ws, cudaStream_t st) {
+  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, ws, st);
+  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, ws, st);
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+const char* dsa_version(void) { return "dsa-b200 0.1 (sm_100a)"; }
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case DSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_DEVICE_INDEX: return "device: out-of-range index skipped";
+    case DSA_ERR_DEVICE_TIMEOUT: return "device: bounded wait gave up";
+    case DSA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+  }
+  return "unknown status";
+}
+
+const char* dsa_last_error(void) { return g_last_error; }
+
+size_t dsa_workspace_size(int op, const dsa_batch* batch, int32_t k, int32_t h_i, int32_t d_i) {
+  (void)h_i;
+  (void)d_i;
+  if (!batch || batch->num_q <= 0 || k <= 0) return 0;
+  const int T = batch->num_q;
+  const int sms = num_sms();
+  switch (op) {
+    case DSA_OP_INDEXER_SCORES:
+    case DSA_OP_TOPK:
+      return 0;
+    case DSA_OP_SPARSE_MLA:
+      return mla_ws_bytes(T, 128, 512, k, sms);
+    case DSA_OP_FUSED_DECODE:
+      return align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float)) +
+             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes(T, 128, 512, k, sms);
+    default:
+      return 0;
+  }
+}
+
+dsa_status dsa_indexer_scores(const dsa_batch* batch, const dsa_indexer_in* in, float* scores, int64_t score_ld,
+                              void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  dsa_status s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_indexer(batch, in)) != DSA_OK) return s;
+  if (!scores) return fail(DSA_ERR_INVALID_ARGUMENT, "scores is NULL");
+  if (score_ld < batch->max_seq_len) return fail(DSA_ERR_INVALID_ARGUMENT, "score_ld < max_seq_len");
+  if (batch->num_q == 0) return DSA_OK;
+  return launch_indexer(batch, in, scores, score_ld, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t score_ld, int32_t k, int32_t* idx,
+                    void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  (void)ws;
+  (void)ws_bytes;
+  dsa_status s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if (!scores || !idx) return fail(DSA_ERR_INVALID_ARGUMENT, "scores and idx must be non-NULL");
+  if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
+  if (score_ld < batch->max_seq_len) return fail(DSA_ERR_INVALID_ARGUMENT, "score_ld < max_seq_len");
+  if (batch->num_q == 0) return DSA_OK;
+  return launch_topk(batch, scores, score_ld, k, idx, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_mla_attn(const dsa_batch* batch, const dsa_mla_in* in, const int32_t* idx, int32_t k,
+                               void* out, float* lse, void* ws, size_t ws_bytes, dsa_stream_t stream) {
+  dsa_status s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_mla(in)) != DSA_OK) return s;
+  if (!idx || !out) return fail(DSA_ERR_INVALID_ARGUMENT, "idx and out must be non-NULL");
+  if (!aligned16(out) || !aligned16(idx)) return fail(DSA_ERR_MISALIGNED, "idx and out must be 16-byte aligned");
+  if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
+  if (batch->num_q == 0) return DSA_OK;
+  const size_t need = mla_ws_bytes(batch->num_q, in->n_heads, in->d_latent, k, num_sms());
+  if (need > 0 && (!ws || ws_bytes < need))
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
+  if (need > 0 && !aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  return launch_mla(batch, in, idx, k, out, lse, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in, const dsa_mla_in* mla_in,
+                            int32_t k, void* out, float* lse, int32_t* idx_out, void* ws, size_t ws_bytes,
+                            const dsa_event_t* stage_events, dsa_stream_t stream) {
+  dsa_status s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_indexer(batch, idx_in)) != DSA_OK) return s;
+  if ((s = check_mla(mla_in)) != DSA_OK) return s;
+  if (!out) return fail(DSA_ERR_INVALID_ARGUMENT, "out is NULL");
+  if (!aligned16(out) || (idx_out && !aligned16(idx_out)))
+    return fail(DSA_ERR_MISALIGNED, "out and idx_out must be 16-byte aligned");
+  if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
+  if (batch->num_q == 0) return DSA_OK;
+  const int T = batch->num_q;
+  const size_t sc_bytes = align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float));
+  const size_t id_bytes = align256(static_cast<size_t>(T) * k * sizeof(int32_t));
+  const size_t mla_bytes = mla_ws_bytes(T, mla_in->n_heads, mla_in->d_latent, k, num_sms());
+  const size_t need = sc_bytes + id_bytes + mla_bytes;
+  if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
+  if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(ws);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sc_bytes);
+  void* mla_ws = static_cast<uint8_t*>(ws) + sc_bytes + id_bytes;
+  auto rec = [&](int i) -> dsa_status {
+    if (!stage_events) return DSA_OK;
+    const cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), st);
+    return e == cudaSuccess ? DSA_OK : fail(DSA_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
+  };
+  if ((s = rec(0)) != DSA_OK) return s;
+  if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st)) != DSA_OK) return s;
+  if ((s = rec(1)) != DSA_OK) return s;
+  if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st)) != DSA_OK) return s;
+  if ((s = rec(2)) != DSA_OK) return s;
+  if ((s = launch_mla(batch, mla_in, idx, k, out, lse, mla_ws, st)) != DSA_OK) return s;
+  return rec(3);
+}
+
+dsa_status dsa_quantize_index_keys(const void* k_bf16, int64_t n_keys, int32_t dim, int32_t group, uint8_t* k8,
+                                   float* scale, dsa_stream_t stream) {
+  if (!k_bf16 || !k8 || !scale) return fail(DSA_ERR_INVALID_ARGUMENT, "k_bf16, k8, scale must be non-NULL");
+  if (n_keys < 0) return fail(DSA_ERR_INVALID_ARGUMENT, "n_keys < 0");
+  if (group != 32 && group != 64 && group != 128) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "group %d not in {32,64,128}", group);
+  if (dim <= 0 || dim > 1024 || dim % group != 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "dim %d must be a multiple of group and <= 1024", dim);
+  if (!aligned16(k_bf16) || !aligned16(k8) || !aligned16(scale))
+    return fail(DSA_ERR_MISALIGNED, "k_bf16, k8, scale must be 16-byte aligned");
+  if (n_keys == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+  const int64_t blocks64 = (n_keys + 7) / 8;
+  const int blocks = static_cast<int>(blocks64 < sms * 16 ? blocks64 : sms * 16);
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(k_bf16);
+  if (group == 32)
+    quantize_keys_kernel<32><<<blocks, 256, 0, st>>>(k, n_keys, dim, k8, scale);
+  else if (group == 64)
+    quantize_keys_kernel<64><<<blocks, 256, 0, st>>>(k, n_keys, dim, k8, scale);
+  else
+    quantize_keys_kernel<128><<<blocks, 256, 0, st>>>(k, n_keys, dim, k8, scale);
+  return check_launch("quantize_index_keys");
+}
+
+dsa_status dsa_dequantize_index_keys(const uint8_t* k8, const float* scale, int64_t n_keys, int32_t dim,
+                                     int32_t group, float* out, dsa_stream_t stream) {
+  if (!k8 || !scale || !out) return fail(DSA_ERR_INVALID_ARGUMENT, "k8, scale, out must be non-NULL");
+  if (n_keys < 0) return fail(DSA_ERR_INVALID_ARGUMENT, "n_keys < 0");
+  if (group != 32 && group != 64 && group != 128) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "group %d not in {32,64,128}", group);
+  if (dim <= 0 || dim > 1024 || dim % group != 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "dim %d must be a multiple of group and <= 1024", dim);
+  if (!aligned16(k8) || !aligned16(out) || !aligned16(scale))
+    return fail(DSA_ERR_MISALIGNED, "k8, scale, out must be 16-byte aligned");
+  if (n_keys == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = n_keys * dim;
+  const int64_t blocks64 = (n / 4 + 255) / 256;
+  const int sms = num_sms();
+  const int blocks = static_cast<int>(blocks64 < sms * 32 ? blocks64 : sms * 32);
+  dequantize_keys_kernel<<<blocks, 256, 0, st>>>(k8, scale, n, dim, group, out);
+  return check_launch("dequantize_index_keys");
+}
+
+dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t* code_out) {
+  if (!code_out) return fail(DSA_ERR_INVALID_ARGUMENT, "code_out is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, dsa::g_device_status, sizeof(int));
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "reading device status: %s", cudaGetErrorString(e));
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(dsa::g_device_status, &zero, sizeof(int));
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "clearing device status: %s", cudaGetErrorString(e));
+  *code_out = v;
+  return DSA_OK;
+}
+
+}  // extern "C"

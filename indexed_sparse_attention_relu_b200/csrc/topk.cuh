@@ -1,0 +1,164 @@
+// topk.cuh -- per-row Top-K of the indexer scores (radix select).
+//
+// Selection (Top-K step of the Lightning Indexer, section 1 of "Day-0
+// Inference Optimization for a New Sparse Attention Architecture"): the K
+// best positions of row t under the order (score desc, position asc), among
+// its n_valid(t) = min(q_pos + 1, seq_len) causal candidates; fewer than K
+// candidates -> all of them, padded with -1. Output ascending by position.
+//
+// Method: scores map to order-preserving uint32 keys (-0 == +0). One CTA per
+// row finds the K-th largest key tau with four 8-bit most-significant-digit
+// histogram passes (warp-aggregated shared atomics), which also yields
+// `need` = how many keys equal to tau must be taken. A final pass walks the
+// row in position order with two block-wide exclusive scans: the first ranks
+// the keys equal to tau (the lowest positions win), the second places every
+// selected position, so the output comes out sorted with no sort. Rows that
+// fit in shared memory are cached there; longer rows are re-read from L2/HBM
+// on each pass. The result depends only on the scores (bit-deterministic).
+#pragma once
+#include <cub/block/block_scan.cuh>
+
+#include "dsa_common.cuh"
+
+namespace dsa {
+
+struct TopkParams {
+  const float* scores;
+  int64_t ld;
+  const int32_t* cu_q;
+  const int32_t* q_pos;
+  const int32_t* seq_lens;
+  int32_t B;
+  int32_t L_max;
+  int32_t K;
+  int32_t* idx;
+  int32_t cache_cap;  // keys that fit in the dynamic shared-memory cache
+};
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
+  constexpr int IPT = 4;
+  constexpr int CHUNK = THREADS * IPT;
+  using Scan = cub::BlockScan<int, THREADS>;
+  __shared__ typename Scan::TempStorage scan_tmp;
+  __shared__ int hist[256];
+  __shared__ int sel_digit, sel_krem, chunk_total;
+  extern __shared__ uint32_t key_cache[];
+
+  const int t = blockIdx.x;
+  const int b = seq_of_token(p.cu_q, p.B, t);
+  const int len = min(__ldg(p.seq_lens + b), p.L_max);
+  const int n = max(0, min(__ldg(p.q_pos + t) + 1, len));
+  int32_t* out = p.idx + static_cast<int64_t>(t) * p.K;
+  const float* row = p.scores + static_cast<int64_t>(t) * p.ld;
+
+  if (n <= p.K) {
+    for (int i = threadIdx.x; i < p.K; i += THREADS) out[i] = (i < n) ? i : -1;
+    return;
+  }
+
+  const bool cached = n <= p.cache_cap;
+  if (cached) {
+    for (int i = threadIdx.x; i < n; i += THREADS) key_cache[i] = float_order_key(__ldg(row + i));
+    __syncthreads();
+  }
+  auto key_at = [&](int i) -> uint32_t { return cached ? key_cache[i] : float_order_key(__ldg(row + i)); };
+
+  uint32_t prefix = 0u, mask = 0u;
+  int krem = p.K;
+  const int lane = lane_id();
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = threadIdx.x; i < 256; i += THREADS) hist[i] = 0;
+    __syncthreads();
+    // n rounded up to a multiple of 32 so every lane of a warp reaches __match_any_sync
+    const int n_pad = (n + 31) & ~31;
+    for (int i = threadIdx.x; i < n_pad; i += THREADS) {
+      const uint32_t key = (i < n) ? key_at(i) : 0u;
+      const bool mine = (i < n) && ((key & mask) == prefix);
+      const unsigned active = __ballot_sync(0xffffffffu, mine);
+      if (mine) {
+        const uint32_t digit = (key >> shift) & 0xFFu;
+        const unsigned peers = __match_any_sync(active, digit);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l owns bins 255-8l .. 248-8l (descending)
+      int local = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) local += hist[255 - 8 * lane - j];
+      int incl = local;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      const int before = incl - local;
+      if (before < krem && krem <= incl) {
+        int acc = before;
+        for (int j = 0; j < 8; ++j) {
+          const int d = 255 - 8 * lane - j;
+          if (acc + hist[d] >= krem) {
+            sel_digit = d;
+            sel_krem = krem - acc;
+            break;
+          }
+          acc += hist[d];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel_digit) << shift;
+    mask |= 0xFFu << shift;
+    krem = sel_krem;
+    __syncthreads();
+  }
+  const uint32_t tau = prefix;   // the K-th largest key
+  const int need = krem;         // keys equal to tau that are taken (lowest positions)
+
+  int eq_run = 0, out_run = 0;
+#pragma unroll 1
+  for (int base = 0; base < n; base += CHUNK) {
+    const int i0 = base + threadIdx.x * IPT;
+    uint32_t k[IPT];
+    int n_eq = 0;
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) {
+      k[u] = (i0 + u < n) ? key_at(i0 + u) : 0u;
+      n_eq += (i0 + u < n && k[u] == tau) ? 1 : 0;
+    }
+    int eq_before, eq_total;
+    Scan(scan_tmp).ExclusiveSum(n_eq, eq_before, eq_total);
+    __syncthreads();
+    eq_before += eq_run;
+    bool sel[IPT];
+    int n_sel = 0;
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) {
+      const bool valid = i0 + u < n;
+      bool s = valid && k[u] > tau;
+      if (valid && k[u] == tau) {
+        s = eq_before < need;
+        ++eq_before;
+      }
+      sel[u] = s;
+      n_sel += s ? 1 : 0;
+    }
+    int out_before, out_total;
+    Scan(scan_tmp).ExclusiveSum(n_sel, out_before, out_total);
+    __syncthreads();
+    out_before += out_run;
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) {
+      if (sel[u] && out_before < p.K) out[out_before++] = i0 + u;
+    }
+    eq_run += eq_total;
+    out_run += out_total;
+  }
+  (void)chunk_total;
+}
+
+}  // namespace dsa

@@ -1,0 +1,92 @@
+"""Device copies of a seeded workload, ready for the C-ABI calls.
+
+Marshalling only: the arrays of :mod:`.workloads` become torch tensors on a
+CUDA device (bf16 bit patterns reinterpreted, int32 metadata copied). FP8
+index keys are produced on the device by the library's own cache-write step
+(``dsa_quantize_index_keys``), as in serving.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+from .workloads import Workload, bf16_bits
+
+
+def bf16_tensor(x: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(bf16_bits(x).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+@dataclasses.dataclass
+class DeviceWorkload:
+    wl: Workload
+    batch: B.Batch
+    q_idx: torch.Tensor
+    w: torch.Tensor
+    k_cache: torch.Tensor            # bf16 [B, L, dI] or uint8 codes
+    k_scale: Optional[torch.Tensor]  # fp32 [B, L, dI/group] (FP8)
+    k_bf16: Optional[torch.Tensor]   # bf16 keys (kept for the FP8 cache write)
+    q: torch.Tensor
+    kv: torch.Tensor
+
+    def indexer_in(self) -> B.dsa_indexer_in:
+        return B.indexer_in(self.q_idx, self.w, self.k_cache, self.k_scale,
+                            self.wl.scale_group if self.k_scale is not None else None)
+
+    def mla_in(self) -> B.dsa_mla_in:
+        return B.mla_in(self.q, self.kv, self.wl.dc, self.wl.softmax_scale)
+
+
+def _cache_tensor(wl: Workload, tag: str, dev) -> torch.Tensor:
+    """[B, Lmax, dim] bf16 cache; built sequence by sequence when the workload
+    was made without host caches (rows past a sequence's length are zero)."""
+    full = wl.k_idx if tag == "k_idx" else wl.kv
+    if full is not None:
+        return bf16_tensor(full, dev)
+    dim = wl.dI if tag == "k_idx" else wl.D
+    out = torch.zeros((wl.B, wl.Lmax, dim), dtype=torch.bfloat16, device=dev)
+    for b in range(wl.B):
+        n = int(wl.seq_lens[b])
+        if n:
+            out[b, :n] = bf16_tensor(wl.seq_rows(tag, b), dev)
+    return out
+
+
+def to_device(wl: Workload, device="cuda", keep_bf16_keys: bool = False) -> DeviceWorkload:
+    dev = torch.device(device)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+    batch = B.Batch(i32(wl.cu_q), i32(wl.q_pos), i32(wl.seq_lens), wl.Lmax)
+    q_idx = bf16_tensor(wl.q_idx, dev)
+    w = torch.from_numpy(np.ascontiguousarray(wl.w, np.float32)).to(dev)
+    k_bf16 = _cache_tensor(wl, "k_idx", dev)
+    k_scale = None
+    k_cache = k_bf16
+    if wl.key_dtype == "fp8":
+        k_cache = torch.empty(k_bf16.shape, dtype=torch.uint8, device=dev)
+        k_scale = torch.empty(k_bf16.shape[:-1] + (wl.dI // wl.scale_group,), dtype=torch.float32, device=dev)
+        B.dsa_quantize_index_keys(k_bf16, wl.scale_group, k_cache, k_scale)
+        if not keep_bf16_keys:
+            k_bf16 = None
+    q = bf16_tensor(wl.q, dev)
+    kv = _cache_tensor(wl, "kv", dev)
+    return DeviceWorkload(wl, batch, q_idx, w, k_cache, k_scale, k_bf16 if wl.key_dtype == "fp8" else None, q, kv)
+
+
+def subset(dw: DeviceWorkload, rows) -> DeviceWorkload:
+    """The same caches with only the query tokens ``rows`` (sorted) kept."""
+    wl = dw.wl
+    rows = np.asarray(rows, np.int64)
+    b = wl.seq_of_token()[rows]
+    counts = np.bincount(b, minlength=wl.B)
+    cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    dev = dw.q.device
+    r = torch.from_numpy(rows).to(dev)
+    sub_wl = dataclasses.replace(wl, T=len(rows), cu_q=cu, q_pos=wl.q_pos[rows].copy(), q_idx=wl.q_idx[rows],
+                                 w=wl.w[rows], q=wl.q[rows])
+    batch = B.Batch(torch.from_numpy(cu).to(dev), dw.batch.q_pos[r].contiguous(), dw.batch.seq_lens, wl.Lmax)
+    return dataclasses.replace(dw, wl=sub_wl, batch=batch, q_idx=dw.q_idx[r].contiguous(), w=dw.w[r].contiguous(),
+                               q=dw.q[r].contiguous())

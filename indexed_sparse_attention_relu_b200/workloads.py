@@ -45,12 +45,18 @@ _SEEDS = {"c1": 1, "c2": 2, "c3": 3, "c4": 4, "c5": 5, "c5i": 51}
 _BLOCK_ROWS = 4096
 
 
-def bf16_round(x: np.ndarray) -> np.ndarray:
-    """Round fp32 values to the nearest bfloat16 (ties to even); returns fp32."""
+def bf16_round(x: np.ndarray, inplace: bool = False) -> np.ndarray:
+    """Round finite fp32 values to the nearest bfloat16 (ties to even); returns fp32."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return (u.astype(np.uint32) << 16).view(np.float32)
+    if not inplace:
+        x = x.copy()
+    u = x.view(np.uint32)
+    r = u >> 16
+    r &= 1
+    r += 0x7FFF
+    u += r                      # no overflow: finite values are below 0xFF800000
+    u &= np.uint32(0xFFFF0000)
+    return x
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -67,18 +73,42 @@ def _stream(seed: int, tag: str, block: int) -> np.random.Generator:
     return np.random.Generator(np.random.Philox(key=_key(seed, tag), counter=[block, 0, 0, 0]))
 
 
-def _draw_rows(seed: int, tag: str, n_rows: int, row_elems: int, law, row_blocks=None) -> np.ndarray:
-    """Draw an [n_rows, row_elems] fp32 array block by block.
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        import concurrent.futures
+        import os
+        _POOL = concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1))
+    return _POOL
+
+
+def _draw_rows(seed: int, tag: str, n_rows: int, row_elems: int, law, row_blocks=None,
+               round_bf16: bool = False) -> np.ndarray:
+    """Draw an [n_rows, row_elems] fp32 array block by block (threads over blocks).
 
     ``law(gen, shape)`` draws one block. ``row_blocks`` optionally restricts the
-    draw to the listed blocks (the others are left zero)."""
+    draw to the listed blocks (the others are left zero). ``round_bf16`` rounds
+    each block to bfloat16 in place."""
     out = np.zeros((n_rows, row_elems), dtype=np.float32)
     n_blocks = (n_rows + _BLOCK_ROWS - 1) // _BLOCK_ROWS
     blocks = range(n_blocks) if row_blocks is None else sorted(set(row_blocks))
-    for blk in blocks:
+
+    def one(blk):
         r0 = blk * _BLOCK_ROWS
         r1 = min(n_rows, r0 + _BLOCK_ROWS)
         out[r0:r1] = law(_stream(seed, tag, blk), (r1 - r0, row_elems))
+        if round_bf16:
+            bf16_round(out[r0:r1], inplace=True)
+
+    blocks = list(blocks)
+    if len(blocks) > 1:
+        list(_pool().map(one, blocks))
+    else:
+        for blk in blocks:
+            one(blk)
     return out
 
 
@@ -132,6 +162,7 @@ class Workload:
     kv: Optional[np.ndarray]
     seed: int
     integer_valued: bool
+    laws: dict = dataclasses.field(default_factory=dict, repr=False)  # cache tag -> value law
 
     @property
     def D(self) -> int:
@@ -145,6 +176,12 @@ class Workload:
         """Causal candidate count per query: min(pos + 1, len of its sequence)."""
         b = self.seq_of_token()
         return np.minimum(self.q_pos + 1, self.seq_lens[b]).astype(np.int32)
+
+    def seq_rows(self, tag: str, b: int) -> np.ndarray:
+        """Cache rows [seq_len_b, dim] of sequence b (tag 'k_idx' or 'kv'), regenerated
+        from the same counter-based streams the full cache is drawn from."""
+        dim = self.dI if tag == "k_idx" else self.D
+        return _draw_rows(self.seed, f"{tag}/{b}", int(self.seq_lens[b]), dim, self.laws[tag], round_bf16=True)
 
 
 def _cache(seed, tag, B, Lmax, lens, dim, law, rows_needed=None):
@@ -161,9 +198,8 @@ def _cache(seed, tag, B, Lmax, lens, dim, law, rows_needed=None):
             blocks = {int(r) // _BLOCK_ROWS for r in rows}
             if not blocks:
                 continue
-        part = _draw_rows(seed, f"{tag}/{b}", n, dim, law, blocks)
-        out[b, :n] = part
-    return bf16_round(out)
+        out[b, :n] = _draw_rows(seed, f"{tag}/{b}", n, dim, law, blocks, round_bf16=True)
+    return out
 
 
 def make(name: str, *, with_caches: bool = True, rows_needed: Optional[Dict[int, list]] = None,
@@ -237,7 +273,7 @@ def make(name: str, *, with_caches: bool = True, rows_needed: Optional[Dict[int,
                   seq_lens=lens.astype(np.int32), HI=HI, dI=dI, H=H, dc=dc, dr=dr, K=K,
                   key_dtype=key_dtype, scale_group=128 if dI >= 128 else dI,
                   softmax_scale=float(1.0 / np.sqrt(D)), q_idx=q_idx, w=w, k_idx=k_idx, q=q, kv=kv,
-                  seed=seed, integer_valued=integer)
+                  seed=seed, integer_valued=integer, laws={"k_idx": law_k, "kv": law_mla})
     if tokens is not None:
         wl = _select_tokens(wl, tokens)
     return wl
@@ -292,7 +328,34 @@ def scaled(name: str, *, B: int, Lmax: int, T_per_seq: int = 1, lens=None, K: Op
     return Workload(name=f"{name}-scaled", B=B, T=T, Lmax=Lmax, cu_q=cu_q, q_pos=q_pos, seq_lens=lens,
                     HI=HI, dI=dI, H=H, dc=dc, dr=dr, K=K, key_dtype=key_dtype,
                     scale_group=128 if dI >= 128 else dI, softmax_scale=float(1.0 / np.sqrt(D)),
-                    q_idx=q_idx, w=w, k_idx=k_idx, q=q, kv=kv, seed=seed, integer_valued=integer)
+                    q_idx=q_idx, w=w, k_idx=k_idx, q=q, kv=kv, seed=seed, integer_valued=integer,
+                    laws={"k_idx": law_k, "kv": law_mla})
+
+
+def restrict(wl: Workload, rows) -> Workload:
+    """The workload seen by the query tokens ``rows`` only: their sequences
+    (renumbered, in order), caches regenerated for those sequences alone, and
+    Lmax cut to the longest of them. Values are identical to the full
+    workload's: used to run the oracle on sampled rows of very large caches."""
+    rows = np.asarray(rows, np.int64)
+    seqs = np.unique(wl.seq_of_token()[rows])
+    remap = {int(b): i for i, b in enumerate(seqs)}
+    lens = wl.seq_lens[seqs].astype(np.int32)
+    Lmax = int(lens.max())
+    bt = np.array([remap[int(b)] for b in wl.seq_of_token()[rows]], np.int32)
+    order = np.argsort(bt, kind="stable")
+    rows, bt = rows[order], bt[order]
+    counts = np.bincount(bt, minlength=len(seqs))
+    cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    k_idx = np.zeros((len(seqs), Lmax, wl.dI), np.float32)
+    kv = np.zeros((len(seqs), Lmax, wl.D), np.float32)
+    for i, b in enumerate(seqs):
+        n = int(wl.seq_lens[b])
+        k_idx[i, :n] = wl.seq_rows("k_idx", int(b))
+        kv[i, :n] = wl.seq_rows("kv", int(b))
+    return dataclasses.replace(wl, B=len(seqs), T=len(rows), Lmax=Lmax, cu_q=cu, q_pos=wl.q_pos[rows].copy(),
+                               seq_lens=lens, q_idx=wl.q_idx[rows].copy(), w=wl.w[rows].copy(),
+                               q=wl.q[rows].copy(), k_idx=k_idx, kv=kv), rows
 
 
 CONFIGS = tuple(_SEEDS)

@@ -1,0 +1,147 @@
+"""The C-ABI library loads, exports every symbol include/dsa.h declares, and
+rejects bad arguments with a status before anything is enqueued.
+
+These run without a GPU: every call below fails validation, which happens on
+the host before any CUDA call, so fake (never dereferenced) pointers are fine.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from indexed_sparse_attention_relu_b200 import binding as B
+from indexed_sparse_attention_relu_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return B.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(B.EXPORTED) == names
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert B.status_string(s)
+    assert lib.dsa_version().decode().startswith("dsa-b200")
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+MIS = 0x10004   # misaligned
+
+
+def _batch(**kw):
+    d = dict(batch=2, num_q=2, max_seq_len=256, cu_q=FAKE, q_pos=FAKE, seq_lens=FAKE, block_table=None, page_size=0)
+    d.update(kw)
+    return B.dsa_batch(**d)
+
+
+def _idx_in(**kw):
+    d = dict(n_heads=64, head_dim=128, q=FAKE, w=FAKE, key_dtype=B.DSA_KEY_BF16, k_cache=FAKE, k_scale=None,
+             scale_group=128)
+    d.update(kw)
+    return B.dsa_indexer_in(**d)
+
+
+def _mla_in(**kw):
+    d = dict(n_heads=128, d_latent=512, d_rope=64, softmax_scale=0.04, q=FAKE, kv=FAKE)
+    d.update(kw)
+    return B.dsa_mla_in(**d)
+
+
+def _scores(lib, batch, inp, scores=FAKE, ld=256):
+    return lib.dsa_indexer_scores(ctypes.byref(batch), ctypes.byref(inp), scores, ld, None, 0, None)
+
+
+def test_indexer_validation(lib):
+    assert lib.dsa_indexer_scores(None, ctypes.byref(_idx_in()), FAKE, 256, None, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(batch=0), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(cu_q=None), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(block_table=FAKE), _idx_in()) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(), _idx_in(n_heads=32)) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(), _idx_in(head_dim=96)) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(), _idx_in(q=MIS)) == B.DSA_ERR_MISALIGNED
+    assert _scores(lib, _batch(), _idx_in(key_dtype=7)) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(), _idx_in(key_dtype=B.DSA_KEY_FP8_E4M3)) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(), _idx_in(key_dtype=B.DSA_KEY_FP8_E4M3, k_scale=FAKE, scale_group=32)) == \
+        B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(), _idx_in(), scores=None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(), _idx_in(), ld=100) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(batch=70000, max_seq_len=40000), _idx_in()) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert "shape" in B.last_error() or "2^31" in B.last_error()
+    # an empty batch is a no-op
+    assert _scores(lib, _batch(num_q=0), _idx_in()) == B.DSA_OK
+
+
+def test_topk_validation(lib):
+    b = _batch()
+    assert lib.dsa_topk(ctypes.byref(b), None, 256, 16, FAKE, None, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, 256, 0, FAKE, None, 0, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, 256, 4096, FAKE, None, 0, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert lib.dsa_topk(ctypes.byref(b), FAKE, 255, 16, FAKE, None, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+
+
+def test_mla_validation(lib):
+    b = _batch()
+
+    def call(inp, idx=FAKE, k=64, out=FAKE, ws=None, ws_bytes=0, batch=b):
+        return lib.dsa_sparse_mla_attn(ctypes.byref(batch), ctypes.byref(inp), idx, k, out, None, ws, ws_bytes, None)
+
+    assert call(_mla_in(d_latent=256)) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert call(_mla_in(n_heads=96)) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert call(_mla_in(n_heads=0)) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert call(_mla_in(kv=MIS)) == B.DSA_ERR_MISALIGNED
+    assert call(_mla_in(softmax_scale=float("nan"))) == B.DSA_ERR_INVALID_ARGUMENT
+    assert call(_mla_in(), idx=None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert call(_mla_in(), out=MIS) == B.DSA_ERR_MISALIGNED
+    assert call(_mla_in(), k=0) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    # two queries, K = 2048: several key splits -> a workspace is required
+    assert call(_mla_in(), k=2048) == B.DSA_ERR_WORKSPACE_TOO_SMALL
+    need = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128)
+    assert need > 0
+    assert call(_mla_in(), k=2048, ws=FAKE, ws_bytes=need - 1) == B.DSA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_fused_and_quant_validation(lib):
+    b = _batch()
+    r = lib.dsa_fused_decode(ctypes.byref(b), ctypes.byref(_idx_in()), ctypes.byref(_mla_in()), 2048, FAKE, None,
+                             None, None, 0, None, None)
+    assert r == B.DSA_ERR_WORKSPACE_TOO_SMALL
+    need = lib.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, ctypes.byref(b), 2048, 64, 128)
+    assert need >= 2 * 256 * 4 + 2 * 2048 * 4
+    q = lib.dsa_quantize_index_keys
+    assert q(None, 10, 128, 128, FAKE, FAKE, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert q(FAKE, 10, 128, 48, FAKE, FAKE, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert q(FAKE, 10, 100, 32, FAKE, FAKE, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert q(MIS, 10, 128, 128, FAKE, FAKE, None) == B.DSA_ERR_MISALIGNED
+    assert q(FAKE, -1, 128, 128, FAKE, FAKE, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert q(FAKE, 0, 128, 128, FAKE, FAKE, None) == B.DSA_OK
+    d = lib.dsa_dequantize_index_keys
+    assert d(FAKE, FAKE, 10, 128, 96, FAKE, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert d(FAKE, FAKE, 0, 128, 128, FAKE, None) == B.DSA_OK
+
+
+def test_workspace_sizes(lib):
+    b = _batch(num_q=32, batch=32, max_seq_len=8192)
+    assert lib.dsa_workspace_size(B.DSA_OP_INDEXER_SCORES, ctypes.byref(b), 2048, 64, 128) == 0
+    assert lib.dsa_workspace_size(B.DSA_OP_TOPK, ctypes.byref(b), 2048, 64, 128) == 0
+    fused = lib.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, ctypes.byref(b), 2048, 64, 128)
+    mla = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128)
+    assert fused == 32 * 8192 * 4 + 32 * 2048 * 4 + mla
+    assert lib.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, None, 2048, 64, 128) == 0
