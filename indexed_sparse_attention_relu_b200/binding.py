@@ -193,6 +193,9 @@ def dsa_fused_decode(batch: Batch, idx_inp: dsa_indexer_in, mla_inp: dsa_mla_in,
         ws_bytes = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 0
     ev = None
     if stage_events is not None:
+        for e in stage_events:
+            if not e.cuda_event:          # torch creates the CUDA event on first record
+                e.record(torch.cuda.current_stream() if stream is None else stream)
         arr = (c_void_p * 4)(*[e.cuda_event for e in stage_events])
         ev = ctypes.cast(arr, c_void_p)
     _check(load().dsa_fused_decode(batch.ref, ctypes.byref(idx_inp), ctypes.byref(mla_inp), k, _ptr(out), _ptr(lse),

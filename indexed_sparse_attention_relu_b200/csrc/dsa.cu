@@ -472,3 +472,4 @@ dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t* code_out) {
 }
 
 }  // extern "C"
+

@@ -213,12 +213,18 @@ def test_mla_small_latent_c1_shapes():
 
 def test_mla_many_tiles_per_split():
     """Many queries -> one key split per query with several 64-key tiles each
-    (the pipelined gather / PV / QK^T order), plus the lazy-rescale path: the
-    later tiles hold keys whose logits grow by far more than 2^8 over the first."""
+    (the pipelined gather / PV / QK^T order), plus the lazy-rescale path: every
+    head's query gets 8 in its first rope dim and the keys at positions >= 600
+    get 32 there (0 before), so later tiles' logits rise uniformly by
+    8 * 32 / sqrt(576) = 10.7 (15.4 in log2 units, above the 2^8 rescale
+    threshold) while the softmax over them stays as flat as before."""
     wl = W.scaled("c2", B=1, Lmax=1200, lens=(1200,), T_per_seq=160, K=640)
+    q = wl.q.copy()
     kv = wl.kv.copy()
-    kv[0, 600:1200, wl.dc:] *= 16.0   # rope dims only: late logits grow ~2^10, values unchanged
-    wl = dataclasses.replace(wl, kv=kv)
+    q[:, :, wl.dc] = 8.0
+    kv[0, :600, wl.dc] = 0.0
+    kv[0, 600:1200, wl.dc] = 32.0
+    wl = dataclasses.replace(wl, kv=kv, q=q)
     nv = wl.n_valid()
     idx = np.full((wl.T, wl.K), -1, np.int32)
     for t in range(wl.T):
