@@ -30,9 +30,9 @@
  *
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers unless stated, row-major, owned
- *    by the caller. The library allocates no device memory, keeps no per-call
- *    state and never synchronises (except dsa_read_device_status), so every
- *    call can be enqueued inside CUDA stream capture.
+ *    by the caller. No call allocates device memory (the one fixed array that
+ *    dsa_fused_decode_noalloc uses is part of the loaded library), keeps
+ *    per-call state or synchronises (except dsa_read_device_status).
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).
  *  - Argument, shape and alignment errors return a status before anything is
  *    enqueued; dsa_last_error() then describes the problem.
@@ -175,6 +175,29 @@ dsa_status dsa_fused_decode(const dsa_batch *batch, const dsa_indexer_in *idx_in
                             const dsa_mla_in *mla_in, int32_t k, void *out, float *lse,
                             int32_t *idx_out, void *ws, size_t ws_bytes,
                             const dsa_event_t *stage_events, dsa_stream_t stream);
+
+/* The decode chain of dsa_fused_decode without a workspace argument, for
+ * callers that cannot provide device memory at call time: for example an
+ * inference runtime or plugin host that reserves all device memory in its own
+ * pool and hands extensions no workspace, or a serving path that must never
+ * enter the CUDA allocator. The paper has no counterpart for this entry
+ * point; it is a service of this library.
+ * Scratch (score rows, and the indices when idx_out is NULL) lives in one
+ * fixed 32 MiB device array inside libdsa.so, held on every device that loads
+ * the library until the process exits. The call allocates and frees nothing.
+ * Limit: num_q * max_seq_len * 4 bytes (+ num_q * k * 4 when idx_out is NULL,
+ * each rounded up to 256) must not exceed 33554432; larger calls return
+ * DSA_ERR_WORKSPACE_TOO_SMALL with the required size in dsa_last_error().
+ * The attention runs with one key split per query, so results agree with
+ * dsa_fused_decode within rounding (indices are identical).
+ * The first call on a device looks up the array's device address with that
+ * device current; make that first call before any stream capture.
+ * All calls share the array: calls whose work overlaps on the GPU (other
+ * streams, other threads) race on it and must be serialised by the caller.
+ * Nothing in the array needs to start at zero; stale contents are never read. */
+dsa_status dsa_fused_decode_noalloc(const dsa_batch *batch, const dsa_indexer_in *idx_in,
+                                    const dsa_mla_in *mla_in, int32_t k, void *out, float *lse,
+                                    int32_t *idx_out, dsa_stream_t stream);
 
 /* Index-key cache write: per-group dynamic FP8 quantisation.
  * k_bf16: bf16 [n_keys, dim]; for every group of `group` elements

@@ -40,7 +40,7 @@ DSA_OP_FUSED_DECODE = 3
 
 # Every symbol include/dsa.h declares.
 EXPORTED = (
-    "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_fused_decode",
+    "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_fused_decode", "dsa_fused_decode_noalloc",
     "dsa_quantize_index_keys", "dsa_dequantize_index_keys", "dsa_workspace_size",
     "dsa_read_device_status", "dsa_status_string", "dsa_last_error", "dsa_version",
 )
@@ -86,6 +86,8 @@ def load() -> ctypes.CDLL:
             "dsa_sparse_mla_attn": (c_int, [POINTER(dsa_batch), POINTER(dsa_mla_in), P, c_int32, P, P, P, c_size_t, P]),
             "dsa_fused_decode": (c_int, [POINTER(dsa_batch), POINTER(dsa_indexer_in), POINTER(dsa_mla_in), c_int32,
                                          P, P, P, P, c_size_t, P, P]),
+            "dsa_fused_decode_noalloc": (c_int, [POINTER(dsa_batch), POINTER(dsa_indexer_in), POINTER(dsa_mla_in),
+                                                 c_int32, P, P, P, P]),
             "dsa_quantize_index_keys": (c_int, [P, c_int64, c_int32, c_int32, P, P, P]),
             "dsa_dequantize_index_keys": (c_int, [P, P, c_int64, c_int32, c_int32, P, P]),
             "dsa_workspace_size": (c_size_t, [c_int, POINTER(dsa_batch), c_int32, c_int32, c_int32]),
@@ -200,6 +202,14 @@ def dsa_fused_decode(batch: Batch, idx_inp: dsa_indexer_in, mla_inp: dsa_mla_in,
         ev = ctypes.cast(arr, c_void_p)
     _check(load().dsa_fused_decode(batch.ref, ctypes.byref(idx_inp), ctypes.byref(mla_inp), k, _ptr(out), _ptr(lse),
                                    _ptr(idx_out), _ptr(ws), ws_bytes, ev, _stream(stream)))
+
+
+def dsa_fused_decode_noalloc(batch: Batch, idx_inp: dsa_indexer_in, mla_inp: dsa_mla_in, k: int,
+                             out: torch.Tensor, lse: torch.Tensor | None = None, idx_out: torch.Tensor | None = None,
+                             stream=None) -> None:
+    """The decode chain with the library's built-in scratch (no workspace)."""
+    _check(load().dsa_fused_decode_noalloc(batch.ref, ctypes.byref(idx_inp), ctypes.byref(mla_inp), k, _ptr(out),
+                                           _ptr(lse), _ptr(idx_out), _stream(stream)))
 
 
 def dsa_quantize_index_keys(k_bf16: torch.Tensor, group: int, k8: torch.Tensor, scale: torch.Tensor,

@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "dsa_common.cuh"
 #include "indexer.cuh"
@@ -473,3 +474,116 @@ dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t* code_out) {
 
 }  // extern "C"
 
+// ============================================================================ allocation-free variant
+//
+// dsa_fused_decode_noalloc runs the same chain as dsa_fused_decode but takes
+// no workspace: its scratch (the fp32 score rows and, when the caller passes
+// no idx_out, the selected indices) lives in one fixed device array compiled
+// into this library. It exists for callers that cannot hand out device
+// memory at call time -- a plugin host or inference runtime that owns every
+// byte of device memory through its own pool and gives extensions no
+// workspace, or a caller on a latency-critical serving path that must never
+// enter the CUDA allocator. The attention runs with one key split per query,
+// so no split-K partials are needed.
+//
+// The array is kNoAllocScratchBytes (32 MiB) on every device that loads the
+// library, held until the process exits. Calls that would need more scratch
+// are rejected. Nothing in it has to start at zero: the indexer writes every
+// score the Top-K reads and the Top-K writes every index the attention
+// reads, so contents left by an earlier call are never used. All calls share
+// the one array: two calls whose work overlaps on the GPU (different streams,
+// or different host threads on one device) race on it and must be ordered by
+// the caller.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. The host-side
+// symbol is only a stand-in, so the address is looked up once per device
+// (with that device current) and cached.
+dsa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(DSA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSA_OK;
+}
+
+// Attention with one key split per query (writes out / lse directly).
+template <int D, int DC>
+dsa_status launch_mla_unsplit_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
+                                float* lse, cudaStream_t st) {
+  using C = MlaCfg<D, DC>;
+  auto kern = sparse_mla_kernel<D, DC>;
+  dsa_status s = set_smem(kern, C::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  MlaParams p;
+  p.cu_q = bt->cu_q;
+  p.seq_lens = bt->seq_lens;
+  p.B = bt->batch;
+  p.L_max = bt->max_seq_len;
+  p.T = bt->num_q;
+  p.H = in->n_heads;
+  p.K = k;
+  p.q = static_cast<const __nv_bfloat16*>(in->q);
+  p.kv = static_cast<const __nv_bfloat16*>(in->kv);
+  p.idx = idx;
+  p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
+  p.keys_per_split = ((k + 63) / 64) * 64;
+  p.splits = 1;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  const int hb = (in->n_heads + 63) / 64;
+  kern<<<dim3(bt->num_q, hb, 1), C::THREADS, C::SMEM_BYTES, st>>>(p);
+  return check_launch("sparse_mla (unsplit)");
+}
+
+}  // namespace
+
+extern "C" dsa_status dsa_fused_decode_noalloc(const dsa_batch* batch, const dsa_indexer_in* idx_in,
+                                               const dsa_mla_in* mla_in, int32_t k, void* out, float* lse,
+                                               int32_t* idx_out, dsa_stream_t stream) {
+  dsa_status s = check_batch(batch);
+  if (s != DSA_OK) return s;
+  if ((s = check_indexer(batch, idx_in)) != DSA_OK) return s;
+  if ((s = check_mla(mla_in)) != DSA_OK) return s;
+  if (!out) return fail(DSA_ERR_INVALID_ARGUMENT, "out is NULL");
+  if (!aligned16(out) || (idx_out && !aligned16(idx_out)))
+    return fail(DSA_ERR_MISALIGNED, "out and idx_out must be 16-byte aligned");
+  if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
+  if (batch->num_q == 0) return DSA_OK;
+  const int T = batch->num_q;
+  const size_t sc_bytes = align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float));
+  const size_t id_bytes = idx_out ? 0 : align256(static_cast<size_t>(T) * k * sizeof(int32_t));
+  if (sc_bytes + id_bytes > kNoAllocScratchBytes)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL,
+                "dsa_fused_decode_noalloc needs %zu bytes of scratch (num_q * max_seq_len * 4%s); its built-in "
+                "array holds %zu bytes",
+                sc_bytes + id_bytes, idx_out ? "" : " + num_q * k * 4", kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != DSA_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(scratch);
+  int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + sc_bytes);
+  if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st)) != DSA_OK) return s;
+  if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st)) != DSA_OK) return s;
+  if (mla_in->d_latent == 512) return launch_mla_unsplit_t<576, 512>(batch, mla_in, idx, k, out, lse, st);
+  return launch_mla_unsplit_t<80, 64>(batch, mla_in, idx, k, out, lse, st);
+}
