@@ -191,6 +191,7 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=8, help="query tokens in the oracle baseline sample")
     ap.add_argument("--ref-tokens", type=int, default=1, help="query tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -236,10 +237,10 @@ def main():
     idx_in = [c.indexer_in() for c in copies]
     mla_in = [c.mla_in() for c in copies]
 
-    def step(i, events=None):
+    def step(i, events=None, st=None):
         j = i % len(copies)
         B.dsa_fused_decode(copies[j].batch, idx_in[j], mla_in[j], K, outs[j], lses[j], None, ws, ws_bytes,
-                           stage_events=events, stream=stream)
+                           stage_events=events, stream=stream if st is None else st)
 
     for i in range(args.warmup):
         step(i)
@@ -251,18 +252,48 @@ def main():
     t_end = torch.cuda.Event(enable_timing=True)
     for e in [x for row in ev for x in row] + [t_start, t_end]:
         e.record(stream)            # creates the CUDA events outside the timed region
+    torch.cuda.synchronize(dev)
+    # The K timed steps are captured once as one CUDA graph and replayed once,
+    # so host launch overhead cannot hide in the device time (every call of
+    # the library is capture-safe: no allocation, no synchronisation).
+    graph = None
+    timing_mode = "eager"
+    if not args.eager:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(dev)
+            with torch.cuda.graph(graph, stream=cap):
+                for i in range(args.steps):
+                    step(i, None, st=cap)
+            timing_mode = "cuda_graph"
+        except Exception as e:  # report and fall back to eager launches
+            graph = None
+            timing_mode = f"eager (graph capture failed: {type(e).__name__})"
+            torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    # timed region: K steps exactly as a caller runs them (programmatic launch
+    # between the kernels, no events in between)
     with ClockSampler(dev) as clocks:
         t_start.record(stream)
-        for i in range(args.steps):
-            step(i, ev[i])
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(args.steps):
+                step(i)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
+    # per-kernel durations: a second pass of K steps, launched eagerly with an
+    # event recorded on the launch stream right before and after each stage
+    # (events inside a graph cannot be timed; an event between two kernels also
+    # turns the programmatic launch off on that edge)
+    for i in range(args.steps):
+        step(i, ev[i])
+    torch.cuda.synchronize(dev)
     stage_ms = {
         "indexer": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
         "topk": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
@@ -324,14 +355,9 @@ def main():
         except Exception:
             traffic = None
 
-    # kernels launched per step: indexer, topk, attention (+ split combine)
-    from indexed_sparse_attention_relu_b200.binding import load
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    tiles = (K + 63) // 64
-    splits = max(1, min(tiles, (sms + T - 1) // T))
-    tps = (tiles + splits - 1) // splits
-    splits = (tiles + tps - 1) // tps
-    launches_per_step = 3 + (1 if splits > 1 else 0)
+    # kernels launched per step: indexer, Top-K, attention (split partials merge
+    # inside a cluster, so there is no separate combine launch)
+    launches_per_step = 3
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -349,10 +375,12 @@ def main():
                           "frac": step_gbs / peak, "frac_of_8TBps": step_gbs / 8000.0,
                           "algorithmic_bytes": algo["step"]},
         "stage_ms": stage_ms,
+        "stage_ms_note": "second K-step pass, eager launches with CUDA events between the stages",
         "clocks": clocks.summary(),
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
+        "timing": timing_mode,
         "device_status": [status, status2],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -69,7 +69,8 @@ typedef enum {
     DSA_ERR_CUDA = 4,               /* a CUDA runtime call or launch failed */
     DSA_ERR_DEVICE_INDEX = 5,       /* device status: an index out of range was skipped */
     DSA_ERR_DEVICE_TIMEOUT = 6,     /* device status: a bounded wait gave up */
-    DSA_ERR_MISALIGNED = 7          /* a pointer is not 16-byte aligned */
+    DSA_ERR_MISALIGNED = 7,         /* a pointer is not 16-byte aligned */
+    DSA_ERR_DEVICE_LAYOUT = 8       /* device status: a kernel found its shared memory misaligned */
 } dsa_status;
 
 typedef enum { DSA_KEY_BF16 = 0, DSA_KEY_FP8_E4M3 = 1 } dsa_key_dtype;
@@ -160,7 +161,10 @@ dsa_status dsa_topk(const dsa_batch *batch, const float *scores, int64_t score_l
  * out: bf16 [T, n_heads, d_latent]:  sum_i softmax_i(scale * q.kv_i) * kv_i[0:d_latent]
  * lse: fp32 [T, n_heads] natural-log sum-exp of the scaled logits, or NULL.
  * A row with no valid index gets out = 0 and lse = -inf.
- * ws: dsa_workspace_size(DSA_OP_SPARSE_MLA, ...) bytes (split-K partials). */
+ * ws: unused (dsa_workspace_size(DSA_OP_SPARSE_MLA, ...) is 0); may be NULL.
+ * Work split: one CTA per (query, 64-head block, key split); the key splits
+ * of a query form a thread-block cluster and merge through distributed
+ * shared memory, so no intermediate goes to global memory. */
 dsa_status dsa_sparse_mla_attn(const dsa_batch *batch, const dsa_mla_in *in, const int32_t *idx,
                                int32_t k, void *out, float *lse, void *ws, size_t ws_bytes,
                                dsa_stream_t stream);

@@ -29,6 +29,7 @@ DSA_ERR_CUDA = 4
 DSA_ERR_DEVICE_INDEX = 5
 DSA_ERR_DEVICE_TIMEOUT = 6
 DSA_ERR_MISALIGNED = 7
+DSA_ERR_DEVICE_LAYOUT = 8
 
 DSA_KEY_BF16 = 0
 DSA_KEY_FP8_E4M3 = 1

@@ -85,6 +85,22 @@ dsa_status make_key_map(CUtensorMap* map, const void* base, int64_t rows, int di
   return DSA_OK;
 }
 
+// 2-D bf16 map with a 128-byte swizzle: x = element within a row (box 64),
+// y = row (box box_rows; 1 for tile::gather4 row gathers).
+dsa_status make_bf16_rows_map(CUtensorMap* map, const void* base, int64_t rows, int cols, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2u};
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled (rows) failed (%d)", static_cast<int>(r));
+  return DSA_OK;
+}
+
 // ---------------------------------------------------------------- validation
 dsa_status check_batch(const dsa_batch* bt) {
   if (!bt) return fail(DSA_ERR_INVALID_ARGUMENT, "batch is NULL");
@@ -142,21 +158,23 @@ struct MlaPlan {
   int keys_per_split;
 };
 
-MlaPlan mla_plan(int T, int K, int sms) {
+// Key splits per (token, head block): enough CTAs to fill the SMs in one
+// wave, at most 8 (the splits of one (token, head block) form a cluster and
+// merge through distributed shared memory).
+MlaPlan mla_plan(int T, int HB, int K, int sms) {
   const int tiles = (K + 63) / 64;
-  int splits = T > 0 ? (sms + T - 1) / T : 1;
-  splits = splits < 1 ? 1 : (splits > tiles ? tiles : splits);
+  const int base = T * HB;
+  int splits = base >= sms ? 1 : sms / base;
+  if (splits > 8) splits = 8;
+  if (splits > tiles) splits = tiles;
+  if (splits < 1) splits = 1;
   const int tps = (tiles + splits - 1) / splits;
   splits = (tiles + tps - 1) / tps;
   return MlaPlan{splits, tps * 64};
 }
 
-size_t mla_ws_bytes(int T, int H, int DC, int K, int sms) {
-  const MlaPlan pl = mla_plan(T, K, sms);
-  if (pl.splits <= 1) return 0;
-  const size_t rows = static_cast<size_t>(pl.splits) * T * H;
-  return align256(rows * DC * sizeof(float)) + align256(rows * sizeof(float));
-}
+// The attention needs no workspace: split partials merge inside a cluster.
+size_t mla_ws_bytes() { return 0; }
 
 // ---------------------------------------------------------------- launches
 template <typename Kern>
@@ -179,11 +197,14 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   const int64_t groups64 = static_cast<int64_t>((bt->num_q + G - 1) / G) + bt->batch;
   const int groups = static_cast<int>(groups64 < bt->num_q ? groups64 : bt->num_q);
   const int max_tiles = (bt->max_seq_len + 127) / 128;
-  int per_group = sms / (groups > 0 ? groups : 1);
-  if (per_group < 1) per_group = 1;
-  int tpc = (max_tiles + per_group - 1) / per_group;
-  if (tpc > 64) tpc = 64;
-  if (tpc < 1) tpc = 1;
+  // Key tiles per CTA: about four CTAs per SM over the whole grid, so the
+  // hardware scheduler balances ragged and causal rows; at least 2 tiles so
+  // the per-CTA prologue stays amortised, at most 64.
+  const int64_t work = static_cast<int64_t>(groups) * max_tiles;
+  int64_t tpc64 = (work + 4LL * sms - 1) / (4LL * sms);
+  if (tpc64 < 2) tpc64 = 2;
+  if (tpc64 > 64) tpc64 = 64;
+  const int tpc = static_cast<int>(tpc64);
   const int gy = (max_tiles + tpc - 1) / tpc;
   IndexerParams p;
   p.cu_q = bt->cu_q;
@@ -223,7 +244,8 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_in* in, float* 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkCacheMax = 49152;  // keys (192 KB)
 
-dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int k, int32_t* idx, cudaStream_t st) {
+dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int k, int32_t* idx, cudaStream_t st,
+                       bool pdl = false) {
   const int cap = bt->max_seq_len < kTopkCacheMax ? bt->max_seq_len : kTopkCacheMax;
   const int bytes = cap * 4;
   dsa_status s = set_smem(topk_kernel<kTopkThreads>, bytes);
@@ -239,19 +261,33 @@ dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int
   p.K = k;
   p.idx = idx;
   p.cache_cap = cap;
-  topk_kernel<kTopkThreads><<<bt->num_q, kTopkThreads, bytes, st>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(bt->num_q);
+  cfg.blockDim = dim3(kTopkThreads);
+  cfg.dynamicSmemBytes = bytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_kernel<kTopkThreads>, p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "topk launch: %s", cudaGetErrorString(e));
   return check_launch("topk");
 }
 
 template <int D, int DC>
 dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
-                        float* lse, void* ws, cudaStream_t st) {
+                        float* lse, cudaStream_t st, const MlaPlan& pl, bool pdl) {
   using C = MlaCfg<D, DC>;
   auto kern = sparse_mla_kernel<D, DC>;
   dsa_status s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   const int T = bt->num_q, H = in->n_heads;
-  const MlaPlan pl = mla_plan(T, k, num_sms());
+  CUtensorMap kvmap, qmap;
+  if ((s = make_bf16_rows_map(&kvmap, in->kv, static_cast<int64_t>(bt->batch) * bt->max_seq_len, D, 1)) != DSA_OK)
+    return s;
+  if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(T) * H, D, 64)) != DSA_OK) return s;
   MlaParams p;
   p.cu_q = bt->cu_q;
   p.seq_lens = bt->seq_lens;
@@ -260,36 +296,44 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   p.T = T;
   p.H = H;
   p.K = k;
-  p.q = static_cast<const __nv_bfloat16*>(in->q);
-  p.kv = static_cast<const __nv_bfloat16*>(in->kv);
   p.idx = idx;
   p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
   p.keys_per_split = pl.keys_per_split;
   p.splits = pl.splits;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
-  p.part_o = nullptr;
-  p.part_lse = nullptr;
-  if (pl.splits > 1) {
-    const size_t rows = static_cast<size_t>(pl.splits) * T * H;
-    p.part_o = static_cast<float*>(ws);
-    p.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + align256(rows * DC * sizeof(float)));
-  }
   const int hb = (H + 63) / 64;
-  kern<<<dim3(T, hb, pl.splits), C::THREADS, C::SMEM_BYTES, st>>>(p);
-  if ((s = check_launch("sparse_mla")) != DSA_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(T, hb, pl.splits);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
   if (pl.splits > 1) {
-    mla_combine_kernel<<<static_cast<unsigned>(static_cast<int64_t>(T) * H), 128, 0, st>>>(
-        p.part_o, p.part_lse, pl.splits, T, H, DC, p.out, lse);
-    if ((s = check_launch("mla_combine")) != DSA_OK) return s;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = pl.splits;
+    ++na;
   }
-  return DSA_OK;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, kvmap, qmap, p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla launch: %s", cudaGetErrorString(e));
+  return check_launch("sparse_mla");
 }
 
 dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
-                      void* ws, cudaStream_t st) {
-  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, ws, st);
-  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, ws, st);
+                      cudaStream_t st, bool pdl = false) {
+  const MlaPlan pl = mla_plan(bt->num_q, (in->n_heads + 63) / 64, k, num_sms());
+  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, st, pl, pdl);
+  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, st, pl, pdl);
 }
 
 }  // namespace
@@ -309,6 +353,7 @@ const char* dsa_status_string(dsa_status s) {
     case DSA_ERR_DEVICE_INDEX: return "device: out-of-range index skipped";
     case DSA_ERR_DEVICE_TIMEOUT: return "device: bounded wait gave up";
     case DSA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case DSA_ERR_DEVICE_LAYOUT: return "device: shared memory window misaligned";
   }
   return "unknown status";
 }
@@ -326,10 +371,10 @@ size_t dsa_workspace_size(int op, const dsa_batch* batch, int32_t k, int32_t h_i
     case DSA_OP_TOPK:
       return 0;
     case DSA_OP_SPARSE_MLA:
-      return mla_ws_bytes(T, 128, 512, k, sms);
+      return mla_ws_bytes();
     case DSA_OP_FUSED_DECODE:
       return align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float)) +
-             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes(T, 128, 512, k, sms);
+             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes();
     default:
       return 0;
   }
@@ -369,12 +414,10 @@ dsa_status dsa_sparse_mla_attn(const dsa_batch* batch, const dsa_mla_in* in, con
   if (!idx || !out) return fail(DSA_ERR_INVALID_ARGUMENT, "idx and out must be non-NULL");
   if (!aligned16(out) || !aligned16(idx)) return fail(DSA_ERR_MISALIGNED, "idx and out must be 16-byte aligned");
   if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
+  (void)ws;
+  (void)ws_bytes;
   if (batch->num_q == 0) return DSA_OK;
-  const size_t need = mla_ws_bytes(batch->num_q, in->n_heads, in->d_latent, k, num_sms());
-  if (need > 0 && (!ws || ws_bytes < need))
-    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
-  if (need > 0 && !aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
-  return launch_mla(batch, in, idx, k, out, lse, ws, reinterpret_cast<cudaStream_t>(stream));
+  return launch_mla(batch, in, idx, k, out, lse, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in, const dsa_mla_in* mla_in,
@@ -392,14 +435,12 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
   const int T = batch->num_q;
   const size_t sc_bytes = align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float));
   const size_t id_bytes = align256(static_cast<size_t>(T) * k * sizeof(int32_t));
-  const size_t mla_bytes = mla_ws_bytes(T, mla_in->n_heads, mla_in->d_latent, k, num_sms());
-  const size_t need = sc_bytes + id_bytes + mla_bytes;
+  const size_t need = sc_bytes + id_bytes + mla_ws_bytes();
   if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
   if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   float* scores = static_cast<float*>(ws);
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + sc_bytes);
-  void* mla_ws = static_cast<uint8_t*>(ws) + sc_bytes + id_bytes;
   auto rec = [&](int i) -> dsa_status {
     if (!stage_events) return DSA_OK;
     const cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), st);
@@ -408,9 +449,13 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
   if ((s = rec(0)) != DSA_OK) return s;
   if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st)) != DSA_OK) return s;
   if ((s = rec(1)) != DSA_OK) return s;
-  if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st)) != DSA_OK) return s;
+  // Programmatic dependent launch on the two internal edges: each kernel's
+  // prologue overlaps the tail of the previous one and waits on the device
+  // for its results. Not used when stage events sit between the kernels.
+  const bool pdl = stage_events == nullptr;
+  if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st, pdl)) != DSA_OK) return s;
   if ((s = rec(2)) != DSA_OK) return s;
-  if ((s = launch_mla(batch, mla_in, idx, k, out, lse, mla_ws, st)) != DSA_OK) return s;
+  if ((s = launch_mla(batch, mla_in, idx, k, out, lse, st, pdl)) != DSA_OK) return s;
   return rec(3);
 }
 
@@ -525,34 +570,11 @@ dsa_status noalloc_scratch(void** out) {
 }
 
 // Attention with one key split per query (writes out / lse directly).
-template <int D, int DC>
-dsa_status launch_mla_unsplit_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
-                                float* lse, cudaStream_t st) {
-  using C = MlaCfg<D, DC>;
-  auto kern = sparse_mla_kernel<D, DC>;
-  dsa_status s = set_smem(kern, C::SMEM_BYTES);
-  if (s != DSA_OK) return s;
-  MlaParams p;
-  p.cu_q = bt->cu_q;
-  p.seq_lens = bt->seq_lens;
-  p.B = bt->batch;
-  p.L_max = bt->max_seq_len;
-  p.T = bt->num_q;
-  p.H = in->n_heads;
-  p.K = k;
-  p.q = static_cast<const __nv_bfloat16*>(in->q);
-  p.kv = static_cast<const __nv_bfloat16*>(in->kv);
-  p.idx = idx;
-  p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
-  p.keys_per_split = ((k + 63) / 64) * 64;
-  p.splits = 1;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.part_o = nullptr;
-  p.part_lse = nullptr;
-  const int hb = (in->n_heads + 63) / 64;
-  kern<<<dim3(bt->num_q, hb, 1), C::THREADS, C::SMEM_BYTES, st>>>(p);
-  return check_launch("sparse_mla (unsplit)");
+dsa_status launch_mla_unsplit(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
+                              float* lse, cudaStream_t st) {
+  const MlaPlan pl{1, ((k + 63) / 64) * 64};
+  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, st, pl, false);
+  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, st, pl, false);
 }
 
 }  // namespace
@@ -584,6 +606,5 @@ extern "C" dsa_status dsa_fused_decode_noalloc(const dsa_batch* batch, const dsa
   int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(static_cast<uint8_t*>(scratch) + sc_bytes);
   if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st)) != DSA_OK) return s;
   if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st)) != DSA_OK) return s;
-  if (mla_in->d_latent == 512) return launch_mla_unsplit_t<576, 512>(batch, mla_in, idx, k, out, lse, st);
-  return launch_mla_unsplit_t<80, 64>(batch, mla_in, idx, k, out, lse, st);
+  return launch_mla_unsplit(batch, mla_in, idx, k, out, lse, st);
 }

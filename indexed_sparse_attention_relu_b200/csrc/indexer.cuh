@@ -47,7 +47,9 @@ struct IndexerCfg {
   static constexpr int TILE_BYTES = 128 * DK * 2;          // bf16 key tile (A operand)
   static constexpr int Q_BYTES = N * DK * 2;               // query tile (B operand)
   static constexpr int U8_TILE = 128 * DIN;                // FP8 staging tile
-  static constexpr int ST = FP8 ? 4 : ((200 * 1024 - Q_BYTES) / TILE_BYTES > 6 ? 6 : (200 * 1024 - Q_BYTES) / TILE_BYTES);
+  // Stages: small enough that two CTAs share an SM when the query tile is
+  // small (decode), so one CTA's prologue / tail overlaps the other's stream.
+  static constexpr int ST = FP8 ? (G == 1 ? 2 : 3) : 3;
   static constexpr int CS = 2;                             // converted bf16 tiles (FP8)
   static constexpr int NACC = 2;                           // TMEM accumulator buffers
   static constexpr int TMEM_COLS = (NACC * N <= 32) ? 32 : (NACC * N <= 64) ? 64 : (NACC * N <= 128) ? 128
@@ -63,18 +65,25 @@ struct IndexerCfg {
   static constexpr int NUM_BARS = 2 * ST + 2 * NACC + 2 * CS + 1;
   static constexpr int OFF_W = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_MISC = OFF_W + G * HI * 4;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
+  // No alignment slack: with no static shared memory the dynamic window
+  // starts 1024-byte aligned (checked at run time, see the kernel prologue).
+  static constexpr int SMEM_BYTES = OFF_MISC + 64;
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, N, false, false);
+  static constexpr int MIN_CTAS = (SMEM_BYTES <= 113 * 1024) ? 2 : 1;  // CTAs per SM the footprint allows
   static_assert(N <= 256, "indexer MMA N must be <= 256");
   static_assert(ST >= 2, "need at least two stages");
 };
 
 template <int HI, int DIN, int G, bool FP8>
-__global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, 1)
+__global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerCfg<HI, DIN, G, FP8>::MIN_CTAS)
     indexer_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerParams p) {
   using C = IndexerCfg<HI, DIN, G, FP8>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw;
+  if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-byte alignment
+    if (threadIdx.x == 0) set_device_status(DSA_ERR_DEVICE_LAYOUT);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;                      // [ST]  TMA -> MMA / converters
   uint64_t* empty = bars + C::ST;             // [ST]  MMA / converters -> TMA
@@ -91,6 +100,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
+  pdl_launch_dependents();  // the Top-K may be scheduled; it waits for these scores
 
   if (threadIdx.x == 0) {
     // Locate this CTA's token group: groups are G consecutive tokens of one sequence.
@@ -265,16 +275,18 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, 1)
 #pragma unroll
       for (int g = 0; g < G; ++g) score[g] = 0.0f;
       if constexpr (C::N <= 64) {
+        // all N columns in flight at once, one wait
+        float v[C::N / 16][16];
 #pragma unroll
-        for (int c = 0; c < C::N; c += 16) {
-          float v[16];
-          tmem_ld16(tmem_base + lane_addr + acc * C::N + c, v);
-          tmem_wait_ld();
+        for (int c = 0; c < C::N / 16; ++c) tmem_ld16(tmem_base + lane_addr + acc * C::N + c * 16, v[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < C::N / 16; ++c) {
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
-            const int col = c + u;
+            const int col = c * 16 + u;
             const int g = col / HI;
-            if (g < G) score[g] = fmaf(w_s[col], fmaxf(v[u], 0.0f), score[g]);
+            if (g < G) score[g] = fmaf(w_s[col], fmaxf(v[c][u], 0.0f), score[g]);
           }
         }
       } else {

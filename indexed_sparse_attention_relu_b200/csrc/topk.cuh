@@ -51,6 +51,8 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
   const int n = max(0, min(__ldg(p.q_pos + t) + 1, len));
   int32_t* out = p.idx + static_cast<int64_t>(t) * p.K;
   const float* row = p.scores + static_cast<int64_t>(t) * p.ld;
+  pdl_launch_dependents();  // the attention may be scheduled; it waits for these indices
+  pdl_wait_prior();         // the indexer's scores (and anything before it) are complete
 
   if (n <= p.K) {
     for (int i = threadIdx.x; i < p.K; i += THREADS) out[i] = (i < n) ? i : -1;
@@ -59,7 +61,22 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
 
   const bool cached = n <= p.cache_cap;
   if (cached) {
-    for (int i = threadIdx.x; i < n; i += THREADS) key_cache[i] = float_order_key(__ldg(row + i));
+    // Batched loads: 8 independent reads in flight per thread before any store,
+    // so the row costs one memory latency, not one per element.
+    constexpr int BATCH = 8;
+    for (int base = 0; base < n; base += THREADS * BATCH) {
+      float v[BATCH];
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const int i = base + u * THREADS + threadIdx.x;
+        v[u] = (i < n) ? __ldg(row + i) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const int i = base + u * THREADS + threadIdx.x;
+        if (i < n) key_cache[i] = float_order_key(v[u]);
+      }
+    }
     __syncthreads();
   }
   auto key_at = [&](int i) -> uint32_t { return cached ? key_cache[i] : float_order_key(__ldg(row + i)); };
@@ -72,16 +89,26 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
     const int shift = 24 - 8 * pass;
     for (int i = threadIdx.x; i < 256; i += THREADS) hist[i] = 0;
     __syncthreads();
-    // n rounded up to a multiple of 32 so every lane of a warp reaches __match_any_sync
-    const int n_pad = (n + 31) & ~31;
-    for (int i = threadIdx.x; i < n_pad; i += THREADS) {
-      const uint32_t key = (i < n) ? key_at(i) : 0u;
-      const bool mine = (i < n) && ((key & mask) == prefix);
-      const unsigned active = __ballot_sync(0xffffffffu, mine);
-      if (mine) {
-        const uint32_t digit = (key >> shift) & 0xFFu;
-        const unsigned peers = __match_any_sync(active, digit);
-        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+    // Every lane of a warp runs the same trip count (THREADS is a multiple of
+    // 32), so all lanes reach __ballot_sync / __match_any_sync together.
+    constexpr int HB = 4;
+    for (int base = 0; base < n; base += THREADS * HB) {
+      uint32_t kk[HB];
+#pragma unroll
+      for (int u = 0; u < HB; ++u) {
+        const int i = base + u * THREADS + threadIdx.x;
+        kk[u] = (i < n) ? key_at(i) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < HB; ++u) {
+        const int i = base + u * THREADS + threadIdx.x;
+        const bool mine = (i < n) && ((kk[u] & mask) == prefix);
+        const unsigned active = __ballot_sync(0xffffffffu, mine);
+        if (mine) {
+          const uint32_t digit = (kk[u] >> shift) & 0xFFu;
+          const unsigned peers = __match_any_sync(active, digit);
+          if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
+        }
       }
     }
     __syncthreads();

@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_status_strings(lib):
-    for s in range(8):
+    for s in range(9):
         assert B.status_string(s)
     assert lib.dsa_version().decode().startswith("dsa-b200")
 
@@ -111,11 +111,9 @@ def test_mla_validation(lib):
     assert call(_mla_in(), idx=None) == B.DSA_ERR_INVALID_ARGUMENT
     assert call(_mla_in(), out=MIS) == B.DSA_ERR_MISALIGNED
     assert call(_mla_in(), k=0) == B.DSA_ERR_UNSUPPORTED_SHAPE
-    # two queries, K = 2048: several key splits -> a workspace is required
-    assert call(_mla_in(), k=2048) == B.DSA_ERR_WORKSPACE_TOO_SMALL
-    need = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128)
-    assert need > 0
-    assert call(_mla_in(), k=2048, ws=FAKE, ws_bytes=need - 1) == B.DSA_ERR_WORKSPACE_TOO_SMALL
+    assert call(_mla_in(), k=4096) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    # split partials merge inside a cluster: the attention takes no workspace
+    assert lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128) == 0
 
 
 def test_fused_and_quant_validation(lib):
