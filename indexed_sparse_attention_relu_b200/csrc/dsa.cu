@@ -244,12 +244,28 @@ dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_in* in, float* 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkCacheMax = 49152;  // keys (192 KB)
 
+template <typename Kern>
+dsa_status launch_topk_kernel(Kern kern, int threads, int smem, const TopkParams& p, int rows, cudaStream_t st,
+                              bool pdl) {
+  dsa_status s = set_smem(kern, smem);
+  if (s != DSA_OK) return s;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(rows);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "topk launch: %s", cudaGetErrorString(e));
+  return check_launch("topk");
+}
+
 dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int k, int32_t* idx, cudaStream_t st,
                        bool pdl = false) {
-  const int cap = bt->max_seq_len < kTopkCacheMax ? bt->max_seq_len : kTopkCacheMax;
-  const int bytes = cap * 4;
-  dsa_status s = set_smem(topk_kernel<kTopkThreads>, bytes);
-  if (s != DSA_OK) return s;
   TopkParams p;
   p.scores = scores;
   p.ld = ld;
@@ -260,20 +276,24 @@ dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int
   p.L_max = bt->max_seq_len;
   p.K = k;
   p.idx = idx;
+  const int L = bt->max_seq_len;
+  // rows of up to 1024 * IPT candidates: register/shared-memory resident select
+  if (L <= 1024 * 8) {
+    p.cache_cap = 1024 * 8;
+    return launch_topk_kernel(topk_row_kernel<1024, 8>, 1024, 1024 * 8 * 4, p, bt->num_q, st, pdl);
+  }
+  if (L <= 1024 * 16) {
+    p.cache_cap = 1024 * 16;
+    return launch_topk_kernel(topk_row_kernel<1024, 16>, 1024, 1024 * 16 * 4, p, bt->num_q, st, pdl);
+  }
+  if (L <= 1024 * 32) {
+    p.cache_cap = 1024 * 32;
+    return launch_topk_kernel(topk_row_kernel<1024, 32>, 1024, 1024 * 32 * 4, p, bt->num_q, st, pdl);
+  }
+  // longer rows: multi-pass select streaming the row from L2 / HBM
+  const int cap = L < kTopkCacheMax ? L : kTopkCacheMax;
   p.cache_cap = cap;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(bt->num_q);
-  cfg.blockDim = dim3(kTopkThreads);
-  cfg.dynamicSmemBytes = bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, topk_kernel<kTopkThreads>, p);
-  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "topk launch: %s", cudaGetErrorString(e));
-  return check_launch("topk");
+  return launch_topk_kernel(topk_kernel<kTopkThreads>, kTopkThreads, cap * 4, p, bt->num_q, st, pdl);
 }
 
 template <int D, int DC>
@@ -284,9 +304,7 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   dsa_status s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   const int T = bt->num_q, H = in->n_heads;
-  CUtensorMap kvmap, qmap;
-  if ((s = make_bf16_rows_map(&kvmap, in->kv, static_cast<int64_t>(bt->batch) * bt->max_seq_len, D, 1)) != DSA_OK)
-    return s;
+  CUtensorMap qmap;
   if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(T) * H, D, 64)) != DSA_OK) return s;
   MlaParams p;
   p.cu_q = bt->cu_q;
@@ -324,7 +342,8 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, kvmap, qmap, p);
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(in->kv), qmap, p);
   if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla launch: %s", cudaGetErrorString(e));
   return check_launch("sparse_mla");
 }

@@ -102,40 +102,62 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   const int lane = lane_id();
   pdl_launch_dependents();  // the Top-K may be scheduled; it waits for these scores
 
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     // Locate this CTA's token group: groups are G consecutive tokens of one sequence.
-    int g = blockIdx.x, b = -1;
-    for (int bb = 0; bb < p.B; ++bb) {
-      const int nq = __ldg(p.cu_q + bb + 1) - __ldg(p.cu_q + bb);
-      const int ng = (nq + G - 1) / G;
-      if (g < ng) {
-        b = bb;
-        break;
+    int b = -1, g = blockIdx.x;
+    if constexpr (G == 1) {
+      // one token per group: group index == token index
+      if (static_cast<int>(blockIdx.x) < __ldg(p.cu_q + p.B)) {
+        b = seq_of_token(p.cu_q, p.B, blockIdx.x);
+        g = blockIdx.x - __ldg(p.cu_q + b);
       }
-      g -= ng;
-    }
-    int tb = 0, te = 0, t0 = 0, nt = 0;
-    if (b >= 0) {
-      t0 = __ldg(p.cu_q + b) + g * G;
-      nt = min(G, __ldg(p.cu_q + b + 1) - t0);
-      const int len = min(__ldg(p.seq_lens + b), p.L_max);
-      int nk = 0;
-      for (int i = 0; i < G; ++i) {
-        int nv = 0;
-        if (i < nt) nv = max(0, min(__ldg(p.q_pos + t0 + i) + 1, len));
-        misc[7 + i] = nv;
-        nk = max(nk, nv);
+    } else {
+      // warp-parallel scan of groups-per-sequence, 32 sequences per round
+      int before = 0;
+      for (int c = 0; c < p.B && b < 0; c += 32) {
+        const int bb = c + lane;
+        const int ng = (bb < p.B) ? (__ldg(p.cu_q + bb + 1) - __ldg(p.cu_q + bb) + G - 1) / G : 0;
+        int incl = ng;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        const int excl = incl - ng;
+        const unsigned hit = __ballot_sync(0xffffffffu, ng > 0 && static_cast<int>(blockIdx.x) - before >= excl &&
+                                                            static_cast<int>(blockIdx.x) - before < incl);
+        if (hit) {
+          const int src = __ffs(hit) - 1;
+          b = c + src;
+          g = static_cast<int>(blockIdx.x) - before - __shfl_sync(0xffffffffu, excl, src);
+        }
+        before += __shfl_sync(0xffffffffu, incl, 31);
       }
-      const int n_tiles = (nk + 127) / 128;
-      tb = blockIdx.y * p.tiles_per_cta;
-      te = min(n_tiles, tb + p.tiles_per_cta);
     }
-    misc[0] = b;
-    misc[1] = t0;
-    misc[2] = nt;
-    misc[3] = tb;
-    misc[4] = te;
-    misc[6] = 0;
+    if (lane == 0) {
+      int tb = 0, te = 0, t0 = 0, nt = 0;
+      if (b >= 0) {
+        t0 = __ldg(p.cu_q + b) + g * G;
+        nt = min(G, __ldg(p.cu_q + b + 1) - t0);
+        const int len = min(__ldg(p.seq_lens + b), p.L_max);
+        int nk = 0;
+        for (int i = 0; i < G; ++i) {
+          int nv = 0;
+          if (i < nt) nv = max(0, min(__ldg(p.q_pos + t0 + i) + 1, len));
+          misc[7 + i] = nv;
+          nk = max(nk, nv);
+        }
+        const int n_tiles = (nk + 127) / 128;
+        tb = blockIdx.y * p.tiles_per_cta;
+        te = min(n_tiles, tb + p.tiles_per_cta);
+      }
+      misc[0] = b;
+      misc[1] = t0;
+      misc[2] = nt;
+      misc[3] = tb;
+      misc[4] = te;
+      misc[6] = 0;
+    }
   }
   __syncthreads();
   const int b = misc[0];

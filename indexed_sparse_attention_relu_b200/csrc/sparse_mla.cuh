@@ -10,10 +10,12 @@
 //
 // One CTA = (token, 64-head block, key split); the key splits of one
 // (token, head block) form a thread-block cluster. Per tile of 64 selected keys:
-//  * a producer warp gathers the 64 rows with TMA tile::gather4 (four rows per
-//    instruction, 128-byte swizzle applied by the tensor map) into a
-//    two-stage ring; an index of -1 or out of range becomes an out-of-bounds
-//    row, which TMA fills with zeros;
+//  * four producer warps gather the 64 rows with 16-byte cp.async straight
+//    into the 128-byte-swizzled K-major layout (one warp instruction moves
+//    512 contiguous bytes of a row, three cover a 1152-byte row); each thread
+//    signals its copies through an asynchronous mbarrier arrival, so the
+//    producers run one tile ahead without blocking; an index of -1 or out of
+//    range zero-fills its row (two-stage ring);
 //  * one thread issues S = Q K^T (M = 64 heads, N = 64 keys, K = D) and
 //    O += P V (M = 64, N = d_c in 256-wide pieces, K = 64 keys) on tcgen05;
 //    the value operand is the same shared-memory tile read as an MN-major
@@ -21,8 +23,9 @@
 //  * with M = 64 an accumulator uses lanes 0-15 of each TMEM sub-partition,
 //    so O (all d_c columns) sits at lane offset 0 and S at lane offset 16 of
 //    the same columns: both fit in one SM's TMEM;
-//  * 4 softmax warps (threads 16-31 hold the S rows, threads 0-15 the O rows
-//    of the same heads) run an online softmax in the exp2 domain with lazy
+//  * 4 softmax warps read S with 16-lane TMEM loads, so all 32 threads work:
+//    thread t holds head rows t/4 and t/4 + 8 of its warp's 16 and 16 of the
+//    64 keys; they run an online softmax in the exp2 domain with lazy
 //    rescaling: O is only rescaled (TMEM load/scale/store) when a row maximum
 //    grows by more than 2^8, which keeps P <= 256 and the result exact;
 //  * P is written as bf16 to shared memory (A operand of the PV product).
@@ -66,7 +69,7 @@ struct MlaCfg {
   static constexpr int N_PV = DC < 256 ? DC : 256;
   static constexpr int PV_MMAS = DC / N_PV;
   static constexpr int TMEM_COLS = DC <= 32 ? 32 : DC <= 64 ? 64 : DC <= 128 ? 128 : DC <= 256 ? 256 : 512;
-  static constexpr int NUM_WARPS = 6;  // 0-3 softmax/epilogue, 4 TMA producer, 5 MMA
+  static constexpr int NUM_WARPS = 9;  // 0-3 softmax/epilogue, 4-7 gather producers, 8 MMA + TMEM owner
   static constexpr int THREADS = NUM_WARPS * 32;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + Q_BYTES;
@@ -74,7 +77,7 @@ struct MlaCfg {
   static constexpr int OFF_BAR = OFF_P + P_BYTES;
   static constexpr int NUM_BARS = 2 * NST + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 32 + 1024;
+  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
   static constexpr int MAX_SPLITS = 8;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(64, TK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(64, N_PV, false, true);
@@ -88,14 +91,14 @@ struct MlaCfg {
 
 template <int D, int DC>
 __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
-    sparse_mla_kernel(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap,
+    sparse_mla_kernel(const __nv_bfloat16* __restrict__ kv, const __grid_constant__ CUtensorMap qmap,
                       const MlaParams p) {
   using C = MlaCfg<D, DC>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* kv_full = bars;             // [NST] TMA -> MMA
-  uint64_t* kv_empty = bars + C::NST;   // [NST] MMA (PV done) -> TMA
+  uint64_t* kv_full = bars;             // [NST] gather producers -> MMA
+  uint64_t* kv_empty = bars + C::NST;   // [NST] MMA (PV done) -> gather producers
   uint64_t* q_full = kv_empty + C::NST; // TMA -> MMA
   uint64_t* s_full = q_full + 1;        // MMA (S ready) -> softmax
   uint64_t* s_empty = s_full + 1;       // softmax (S read) -> MMA
@@ -105,6 +108,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
   uint64_t* ready = drain + 1;          // merge: every CTA of the cluster has finished its loop
   uint64_t* recv = ready + 1;           // merge: every partial row destined here has arrived
   int32_t* misc = reinterpret_cast<int32_t*>(smem + C::OFF_MISC);
+  // misc: [0] TMEM base, [1] abort
   volatile int* abort_flag = misc + 1;
 
   const int t = blockIdx.x;
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
-      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_full[i], 128);  // one asynchronous arrival per producer thread
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(q_full, 1);
@@ -135,10 +139,9 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     mbar_init(recv, 64 * S);
     misc[1] = 0;
     fence_mbar_init();
-    prefetch_tensormap(&kvmap);
     prefetch_tensormap(&qmap);
   }
-  if (warp == 5) {
+  if (warp == 8) {
     tmem_alloc(reinterpret_cast<uint32_t*>(misc), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
   const uint32_t tmem_base = static_cast<uint32_t>(misc[0]);
   const uint32_t tmem_s = tmem_base + (16u << 16);  // S at lane offset 16 (M = 64 layout)
 
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     // the query block is an input of the call, not of the Top-K: load it now
     mbar_arrive_expect_tx(q_full, C::Q_BYTES);
     const uint32_t qs = smem_u32(smem + C::OFF_Q);
@@ -160,48 +163,49 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
   }
   pdl_wait_prior();  // the selected indices (Top-K output) are complete from here on
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ TMA producer (one warp)
-    const int32_t row_base = b * p.L_max;
-    const int32_t oob_row = p.B * p.L_max;  // past the end: TMA zero-fills the row
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ gather producers (4 warps)
+    // warp pw copies rows 16pw .. 16pw+15 of each 64-key tile; for one row the
+    // whole warp issues 16-byte chunks 32 at a time (512 contiguous bytes)
+    constexpr int CPR = C::DP / 8;                // 16-byte chunks per padded row
+    constexpr int ROUNDS = (CPR + 31) / 32;
+    const int pw = warp - 4;
+    const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * D;
+    // index of this lane's row (lanes 0..15), fetched one tile ahead
+    int nxt = (lane < 16 && k_begin + 16 * pw + lane < k_end) ? __ldg(idx_row + k_begin + 16 * pw + lane) : -1;
     int issued = 0;
     for (int it = 0; it < n_tiles; ++it) {
       const int st = it & 1;
+      const int cur = nxt;
+      if (it + 1 < n_tiles) {
+        const int kn = k_begin + (it + 1) * C::TK + 16 * pw + lane;
+        nxt = (lane < 16 && kn < k_end) ? __ldg(idx_row + kn) : -1;
+      }
       if (!mbar_wait_warp(&kv_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
+      const bool ok = cur >= 0 && cur < len;
+      if (lane < 16 && cur != -1 && !ok) set_device_status(DSA_ERR_DEVICE_INDEX);
+      const uint32_t stage = smem_u32(smem + C::OFF_KV + st * C::KV_BYTES);
+#pragma unroll 4
+      for (int rr = 0; rr < 16; ++rr) {
+        const int r = 16 * pw + rr;                         // key slot in the tile
+        const int srow = __shfl_sync(0xffffffffu, ok ? cur : -1, rr);
+        const __nv_bfloat16* src_row = kv_seq + static_cast<int64_t>(srow < 0 ? 0 : srow) * D;
+#pragma unroll
+        for (int q = 0; q < ROUNDS; ++q) {
+          const int c = 32 * q + lane;                      // 16-byte chunk of the row
+          if (c < CPR) {
+            const bool has = srow >= 0 && c * 8 < D;
+            cp_async_16(stage + (c / 8) * C::ATOM_COL + sw128_offset(r, c % 8), has ? src_row + c * 8 : kv,
+                        has ? 16u : 0u);
+          }
+        }
+      }
+      cp_async_arrive_noinc(&kv_full[st]);
       ++issued;
-      const int kb = k_begin + it * C::TK;
-      const int s0 = (kb + lane < k_end) ? __ldg(idx_row + kb + lane) : -1;
-      const int s1 = (kb + 32 + lane < k_end) ? __ldg(idx_row + kb + 32 + lane) : -1;
-      const bool ok0 = s0 >= 0 && s0 < len, ok1 = s1 >= 0 && s1 < len;
-      if ((s0 != -1 && !ok0) || (s1 != -1 && !ok1)) set_device_status(DSA_ERR_DEVICE_INDEX);
-      const int32_t r0 = ok0 ? row_base + s0 : oob_row;
-      const int32_t r1 = ok1 ? row_base + s1 : oob_row;
-      if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], C::KV_BYTES);
-      __syncwarp();
-      // lane g < 16 gathers keys 4g .. 4g+3 of the tile
-      int32_t y[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int k = 4 * (lane & 15) + j;  // key slot
-        const int32_t lo = __shfl_sync(0xffffffffu, r0, k & 31);
-        const int32_t hi = __shfl_sync(0xffffffffu, r1, k & 31);
-        y[j] = (k < 32) ? lo : hi;
-      }
-      if (lane < 16) {
-        const uint32_t dst = smem_u32(smem + C::OFF_KV + st * C::KV_BYTES) + lane * 4 * 128;
-#pragma unroll
-        for (int c = 0; c < C::AKQ; ++c)
-          tma_gather4(dst + c * C::ATOM_COL, &kvmap, c * 64, y[0], y[1], y[2], y[3], &kv_full[st]);
-      }
     }
-    // drain: no TMA copy may still be landing when the CTA retires (matters
-    // only after a timeout; otherwise every phase below has completed)
-    if (lane == 0) {
-      volatile int never = 0;
-      mbar_wait(q_full, 0, &never);
-      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it) mbar_wait(&kv_full[it & 1], (it >> 1) & 1, &never);
-    }
-  } else if (warp == 5) {
+    cp_async_wait_all();  // nothing may still be landing when the CTA retires
+    (void)issued;
+  } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_base = smem_u32(smem + C::OFF_Q);
@@ -220,6 +224,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
       // tile it+1 only waits for PV(it-1), which is issued before S(it+1).
       bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
       if (ok) {
+        fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor core reads
         tc_fence_after();
         issue_s(0);
       }
@@ -244,6 +249,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         if (it + 1 < n_tiles) {
           if (!(ok = mbar_wait(s_empty, it & 1, abort_flag))) break;
           if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1, abort_flag))) break;
+          fence_proxy_async_smem();
           tc_fence_after();
           issue_s(it + 1);
         }
@@ -258,96 +264,135 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(sw * 32) << 16;
     const bool is_s = lane >= 16;                          // threads 16..31 own S rows
     const int h_local = sw * 16 + (lane & 15);             // head row inside the block
-    float m_used = -INFINITY;                              // running max (log2 domain)
-    float l = 0.0f;                                        // running sum of P
+    // Rows of S this thread handles in the 16-lane layout: head rows ra, ra+8
+    // of the warp's 16 (h_local = sw*16 + row) and key columns 8j + cc, +1.
+    const int ra = lane >> 2;
+    const int cc = 2 * (lane & 3);
+    float m_a = -INFINITY, m_b = -INFINITY;  // running max per row (log2 domain)
+    float l_a = 0.0f, l_b = 0.0f;            // this thread's share of the running sums
     bool ok = true;
     uint8_t* p_tile = smem + C::OFF_P;
+    // indices of the next tile (for the validity mask), one tile ahead
+    int i0n = (k_begin + lane < k_end) ? __ldg(idx_row + k_begin + lane) : -1;
+    int i1n = (k_begin + 32 + lane < k_end) ? __ldg(idx_row + k_begin + 32 + lane) : -1;
     for (int it = 0; it < n_tiles; ++it) {
-      if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
-      tc_fence_after();
-      float s[64];
-      {
-        float v[4][16];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld16(tmem_base + lane_addr + c * 16, v[c]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int u = 0; u < 16; ++u) s[c * 16 + u] = v[c][u];
+      const int i0 = i0n, i1 = i1n;
+      if (it + 1 < n_tiles) {
+        const int kn = k_begin + (it + 1) * C::TK;
+        i0n = (kn + lane < k_end) ? __ldg(idx_row + kn + lane) : -1;
+        i1n = (kn + 32 + lane < k_end) ? __ldg(idx_row + kn + 32 + lane) : -1;
       }
-      // validity of the 64 keys of this tile (same for every head)
-      const int kb = k_begin + it * C::TK;
-      const int i0 = (kb + lane < k_end) ? __ldg(idx_row + kb + lane) : -1;
-      const int i1 = (kb + 32 + lane < k_end) ? __ldg(idx_row + kb + 32 + lane) : -1;
       const unsigned v0 = __ballot_sync(0xffffffffu, i0 >= 0 && i0 < len);
       const unsigned v1 = __ballot_sync(0xffffffffu, i1 >= 0 && i1 < len);
-      float mt = -INFINITY;
+      if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      float v[32];
+      tmem_ld16x256_x8(tmem_s + lane_addr, v);
+      tmem_wait_ld();
+      // v[4j + 0/1] = row ra, cols 8j+cc, +1; v[4j + 2/3] = row ra+8, same cols
+      float ta = -INFINITY, tb = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) {
-        const bool valid = (j < 32) ? ((v0 >> j) & 1u) : ((v1 >> (j - 32)) & 1u);
-        s[j] = valid ? s[j] * p.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[j]);
-      }
-      float factor = 1.0f;
-      bool need = false;
-      if (is_s) {
-        const float m_new = fmaxf(m_used, mt);
-        need = m_new > m_used + 8.0f;
-        if (need) {
-          factor = exp2f(m_used - m_new);
-          l *= factor;
-          m_used = m_new;
+      for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = 8 * j + cc + e;
+          const bool valid = (col < 32) ? ((v0 >> col) & 1u) : ((v1 >> (col - 32)) & 1u);
+          v[4 * j + e] = valid ? v[4 * j + e] * p.scale_log2 : -INFINITY;
+          v[4 * j + 2 + e] = valid ? v[4 * j + 2 + e] * p.scale_log2 : -INFINITY;
+          ta = fmaxf(ta, v[4 * j + e]);
+          tb = fmaxf(tb, v[4 * j + 2 + e]);
         }
       }
+      ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 1));
+      ta = fmaxf(ta, __shfl_xor_sync(0xffffffffu, ta, 2));
+      tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 1));
+      tb = fmaxf(tb, __shfl_xor_sync(0xffffffffu, tb, 2));
+      float fa = 1.0f, fb = 1.0f;
+      const float na = fmaxf(m_a, ta), nb = fmaxf(m_b, tb);
+      const bool need_a = na > m_a + 8.0f, need_b = nb > m_b + 8.0f;
+      if (need_a) {
+        fa = ex2_approx(m_a - na);  // 0 when m_a = -inf
+        l_a *= fa;
+        m_a = na;
+      }
+      if (need_b) {
+        fb = ex2_approx(m_b - nb);
+        l_b *= fb;
+        m_b = nb;
+      }
       bool o_waited = false;
-      if (__any_sync(0xffffffffu, need && it > 0)) {
-        // O already holds earlier tiles: wait for PV(it-1), then rescale those rows.
+      if (__any_sync(0xffffffffu, (need_a || need_b) && it > 0)) {
+        // O already holds earlier tiles: wait for PV(it-1), then rescale those rows
         if (!(ok = mbar_wait_warp(o_done, (it - 1) & 1, abort_flag))) break;
         o_waited = true;
         tc_fence_after();
-        const float fo = __shfl_sync(0xffffffffu, factor, lane | 16);
+        // O row r (lanes 0..15 in the 32-lane layout) is row ra of thread 4(r%8) (a if r < 8, else b)
+        const int src = 4 * (lane & 7);
+        const float ga = __shfl_sync(0xffffffffu, fa, src);
+        const float gb = __shfl_sync(0xffffffffu, fb, src);
+        const float fo = (lane < 8) ? ga : gb;
         for (int c = 0; c < DC; c += 16) {
-          float v[16];
-          tmem_ld16(tmem_base + lane_addr + c, v);
+          float o[16];
+          tmem_ld16(tmem_base + lane_addr + c, o);
           tmem_wait_ld();
-          if (!is_s) {
+          if (lane < 16) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) v[u] *= fo;
+            for (int u = 0; u < 16; ++u) o[u] *= fo;
           }
-          tmem_st16(tmem_base + lane_addr + c, v);
+          tmem_st16(tmem_base + lane_addr + c, o);
         }
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_empty);
-      // P = 2^(s - m) in bf16; l sums the rounded values actually used by PV
-      uint32_t packed[32];
+      // P = 2^(s - m) in bf16; the sums add the rounded values PV actually uses
+      uint32_t pa[8], pb[8];
 #pragma unroll
-      for (int j = 0; j < 64; j += 2) {
-        const float a = (s[j] == -INFINITY || m_used == -INFINITY) ? 0.0f : exp2f(s[j] - m_used);
-        const float c2 = (s[j + 1] == -INFINITY || m_used == -INFINITY) ? 0.0f : exp2f(s[j + 1] - m_used);
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(a, c2);
-        l += __low2float(pr) + __high2float(pr);
-        packed[j / 2] = *reinterpret_cast<const uint32_t*>(&pr);
+      for (int j = 0; j < 8; ++j) {
+        const float a0 = (m_a == -INFINITY) ? 0.0f : ex2_approx(v[4 * j] - m_a);
+        const float a1 = (m_a == -INFINITY) ? 0.0f : ex2_approx(v[4 * j + 1] - m_a);
+        const float b0 = (m_b == -INFINITY) ? 0.0f : ex2_approx(v[4 * j + 2] - m_b);
+        const float b1 = (m_b == -INFINITY) ? 0.0f : ex2_approx(v[4 * j + 3] - m_b);
+        const __nv_bfloat162 qa = __floats2bfloat162_rn(a0, a1);
+        const __nv_bfloat162 qb = __floats2bfloat162_rn(b0, b1);
+        l_a += __low2float(qa) + __high2float(qa);
+        l_b += __low2float(qb) + __high2float(qb);
+        pa[j] = *reinterpret_cast<const uint32_t*>(&qa);
+        pb[j] = *reinterpret_cast<const uint32_t*>(&qb);
       }
       if (it > 0 && !o_waited) {
         if (!(ok = mbar_wait_warp(o_done, (it - 1) & 1, abort_flag))) break;  // P buffer free
       }
-      if (is_s) {
+      {
+        const int ha = sw * 16 + ra, hb = ha + 8;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(p_tile + sw128_offset(h_local, c)) =
-              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        for (int j = 0; j < 8; ++j) {
+          *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(ha, j) + 2 * cc) = pa[j];
+          *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(hb, j) + 2 * cc) = pb[j];
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
+    // full row sums: add the four threads sharing each row
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    // hand (max, sum) of head row r to O lane r (the 32-lane layout below)
+    float m_used, l;
+    {
+      const int src = 4 * (lane & 7);
+      const float xa = __shfl_sync(0xffffffffu, m_a, src), xb = __shfl_sync(0xffffffffu, m_b, src);
+      const float ya = __shfl_sync(0xffffffffu, l_a, src), yb = __shfl_sync(0xffffffffu, l_b, src);
+      m_used = ((lane & 15) < 8) ? xa : xb;
+      l = ((lane & 15) < 8) ? ya : yb;
+    }
     if (ok) ok = mbar_wait_warp(o_done, (n_tiles - 1) & 1, abort_flag);
-    const float l_h = __shfl_sync(0xffffffffu, l, lane | 16);
-    const float m_h = __shfl_sync(0xffffffffu, m_used, lane | 16);
+    const float l_h = l;        // lane r < 16 owns O row r; lanes 16..31 mirror it
+    const float m_h = m_used;
     const int h = h0 + h_local;
     if (ok) tc_fence_after();
     if (S == 1) {
@@ -458,7 +503,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }

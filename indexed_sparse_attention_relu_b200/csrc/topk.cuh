@@ -188,4 +188,162 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
   (void)chunk_total;
 }
 
+// ---------------------------------------------------------------------------
+// Rows of up to THREADS * IPT candidates (decode and most prefill rows).
+// Thread i owns the contiguous positions [i*IPT, (i+1)*IPT): its keys are
+// cached in shared memory, every radix pass adds into a per-warp histogram
+// (conflicts only inside a warp), 256 threads reduce and scan the 256 bins in
+// parallel, and the final emission needs just two block-wide scans because
+// ownership is already in position order.
+template <int THREADS, int IPT>
+__global__ void __launch_bounds__(THREADS, 1) topk_row_kernel(const TopkParams p) {
+  static_assert(IPT % 4 == 0, "IPT must be a multiple of 4");
+  constexpr int WARPS = THREADS / 32;
+  using Scan = cub::BlockScan<int, THREADS>;
+  __shared__ typename Scan::TempStorage scan_tmp;
+  __shared__ int whist[WARPS][256];
+  __shared__ int wsum[8];
+  __shared__ int sel_digit, sel_krem;
+  extern __shared__ __align__(16) uint32_t keys[];  // THREADS * IPT
+
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = lane_id();
+  const int warp = warp_id();
+  const int b = seq_of_token(p.cu_q, p.B, t);
+  const int len = min(__ldg(p.seq_lens + b), p.L_max);
+  const int n = max(0, min(__ldg(p.q_pos + t) + 1, len));
+  int32_t* out = p.idx + static_cast<int64_t>(t) * p.K;
+  const float* row = p.scores + static_cast<int64_t>(t) * p.ld;
+  pdl_launch_dependents();
+  pdl_wait_prior();
+
+  if (n <= p.K) {
+    for (int i = tid; i < p.K; i += THREADS) out[i] = (i < n) ? i : -1;
+    return;
+  }
+  for (int i = tid; i < WARPS * 256; i += THREADS) (&whist[0][0])[i] = 0;
+
+  // ---- load this thread's contiguous positions (all loads in flight at once)
+  const int base = tid * IPT;
+  {
+    float v[IPT];
+    const bool vec = ((p.ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(p.scores) & 15) == 0);
+    if (vec && base + IPT <= n) {
+#pragma unroll
+      for (int u = 0; u < IPT; u += 4) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(row + base + u));
+        v[u] = f.x;
+        v[u + 1] = f.y;
+        v[u + 2] = f.z;
+        v[u + 3] = f.w;
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < IPT; ++u) v[u] = (base + u < n) ? __ldg(row + base + u) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < IPT; u += 4) {
+      uint4 k4;
+      k4.x = (base + u + 0 < n) ? float_order_key(v[u + 0]) : 0u;
+      k4.y = (base + u + 1 < n) ? float_order_key(v[u + 1]) : 0u;
+      k4.z = (base + u + 2 < n) ? float_order_key(v[u + 2]) : 0u;
+      k4.w = (base + u + 3 < n) ? float_order_key(v[u + 3]) : 0u;
+      *reinterpret_cast<uint4*>(keys + base + u) = k4;
+    }
+  }
+  const int mine = max(0, min(IPT, n - base));  // valid positions owned by this thread
+  __syncthreads();
+
+  uint32_t prefix = 0u, mask = 0u;
+  int krem = p.K;
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+#pragma unroll
+    for (int u = 0; u < IPT; u += 4) {
+      const uint4 k4 = *reinterpret_cast<const uint4*>(keys + base + u);
+      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (u + j < mine && (kk[j] & mask) == prefix) atomicAdd(&whist[warp][(kk[j] >> shift) & 0xFFu], 1);
+    }
+    __syncthreads();
+    // 256 threads: bin total (descending digit order), reset, inclusive scan
+    int cnt = 0, incl = 0;
+    if (tid < 256) {
+      const int d = 255 - tid;
+#pragma unroll 4
+      for (int w = 0; w < WARPS; ++w) {
+        cnt += whist[w][d];
+        whist[w][d] = 0;
+      }
+      incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) wsum[warp] = incl;
+    }
+    __syncthreads();
+    if (tid < 256) {
+      int before_warp = 0;
+      for (int w = 0; w < warp; ++w) before_warp += wsum[w];
+      incl += before_warp;
+      const int excl = incl - cnt;
+      if (excl < krem && krem <= incl) {
+        sel_digit = 255 - tid;
+        sel_krem = krem - excl;
+      }
+    }
+    __syncthreads();
+    prefix |= static_cast<uint32_t>(sel_digit) << shift;
+    mask |= 0xFFu << shift;
+    krem = sel_krem;
+  }
+  const uint32_t tau = prefix;   // the K-th largest key
+  const int need = krem;         // keys equal to tau that are taken (lowest positions first)
+
+  int n_eq = 0;
+#pragma unroll
+  for (int u = 0; u < IPT; ++u) n_eq += (u < mine && keys[base + u] == tau) ? 1 : 0;
+  int eq_before, eq_total;
+  Scan(scan_tmp).ExclusiveSum(n_eq, eq_before, eq_total);
+  __syncthreads();
+  int n_sel = 0;
+  {
+    int e = eq_before;
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) {
+      if (u >= mine) break;
+      const uint32_t k = keys[base + u];
+      if (k > tau) {
+        ++n_sel;
+      } else if (k == tau) {
+        n_sel += (e < need) ? 1 : 0;
+        ++e;
+      }
+    }
+  }
+  int out_before, out_total;
+  Scan(scan_tmp).ExclusiveSum(n_sel, out_before, out_total);
+  {
+    int e = eq_before, o = out_before;
+#pragma unroll
+    for (int u = 0; u < IPT; ++u) {
+      if (u >= mine) break;
+      const uint32_t k = keys[base + u];
+      bool take = k > tau;
+      if (k == tau) {
+        take = e < need;
+        ++e;
+      }
+      if (take && o < p.K) out[o++] = base + u;
+    }
+  }
+  (void)eq_total;
+  (void)out_total;
+}
+
 }  // namespace dsa
