@@ -197,14 +197,16 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   const int64_t groups64 = static_cast<int64_t>((bt->num_q + G - 1) / G) + bt->batch;
   const int groups = static_cast<int>(groups64 < bt->num_q ? groups64 : bt->num_q);
   const int max_tiles = (bt->max_seq_len + 127) / 128;
-  // Key tiles per CTA: about four CTAs per SM over the whole grid, so the
-  // hardware scheduler balances ragged and causal rows; at least 2 tiles so
-  // the per-CTA prologue stays amortised, at most 64.
-  const int64_t work = static_cast<int64_t>(groups) * max_tiles;
-  int64_t tpc64 = (work + 4LL * sms - 1) / (4LL * sms);
-  if (tpc64 < 2) tpc64 = 2;
-  if (tpc64 > 64) tpc64 = 64;
-  const int tpc = static_cast<int>(tpc64);
+  // Key tiles per CTA: split each group's key range so the grid fills the
+  // resident CTA slots (C::MIN_CTAS per SM) about once; at least 2 tiles so
+  // the prologue stays amortised, at most 64 (ragged / causal rows then
+  // spread over several CTAs and the hardware scheduler balances them).
+  const int slots = sms * C::MIN_CTAS;
+  int per_group = slots / (groups > 0 ? groups : 1);
+  if (per_group < 1) per_group = 1;
+  int tpc = (max_tiles + per_group - 1) / per_group;
+  if (tpc < 2) tpc = 2;
+  if (tpc > 64) tpc = 64;
   const int gy = (max_tiles + tpc - 1) / tpc;
   IndexerParams p;
   p.cu_q = bt->cu_q;

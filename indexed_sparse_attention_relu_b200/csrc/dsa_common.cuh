@@ -303,6 +303,32 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Brings `bytes` (a multiple of 16) starting at `src` into L2 without using
+// shared memory; no completion is tracked.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Sequence of token t from cu_q[0..B]: one warp, 32 boundaries per round
+// (coalesced) instead of a dependent binary search; every lane gets the answer.
+__device__ __forceinline__ int seq_of_token_warp(const int32_t* __restrict__ cu_q, int B, int t) {
+  const int lane = threadIdx.x & 31;
+  // stride through the boundaries in rounds of 32 until the bracket is found
+  int lo = 0, hi = B;          // answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int span = hi - lo;
+    const int step = (span + 31) / 32;
+    const int pos = lo + lane * step;                    // candidate lower bound
+    const bool le = pos < hi && __ldg(cu_q + pos) <= t;  // cu_q[pos] <= t
+    const unsigned m = __ballot_sync(0xffffffffu, le);
+    const int last = 31 - __clz(m);                      // last lane with cu_q[pos] <= t (lane 0 always)
+    const int nlo = lo + last * step;
+    hi = min(hi, nlo + step);
+    lo = nlo;
+  }
+  return lo;
+}
+
 // Arrives on `bar` once every cp.async issued so far by this thread has landed
 // (the barrier's expected count includes this arrival).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {

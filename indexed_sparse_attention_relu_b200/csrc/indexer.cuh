@@ -102,13 +102,30 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   const int lane = lane_id();
   pdl_launch_dependents();  // the Top-K may be scheduled; it waits for these scores
 
+  // Single-token groups: the query rows depend only on the block index, so
+  // their loads go out before the group lookup and overlap it.
+  constexpr int QCPR = C::DK / 8;                                   // 16-byte chunks per B row
+  constexpr int QPT = (C::N * QCPR + C::THREADS - 1) / C::THREADS;  // chunks per thread
+  uint4 qreg[G == 1 ? QPT : 1];
+  if constexpr (G == 1) {
+    const bool tok_ok = static_cast<int>(blockIdx.x) < __ldg(p.cu_q + p.B);
+#pragma unroll
+    for (int u = 0; u < QPT; ++u) {
+      const int i = threadIdx.x + u * C::THREADS;
+      const int n = i / QCPR, c = i % QCPR;
+      qreg[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (tok_ok && i < C::N * QCPR && n < HI && c * 8 < DIN)
+        qreg[u] = __ldg(reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(blockIdx.x) * HI + n) * DIN + c * 8)));
+    }
+  }
+
   if (warp == 0) {
     // Locate this CTA's token group: groups are G consecutive tokens of one sequence.
     int b = -1, g = blockIdx.x;
     if constexpr (G == 1) {
       // one token per group: group index == token index
       if (static_cast<int>(blockIdx.x) < __ldg(p.cu_q + p.B)) {
-        b = seq_of_token(p.cu_q, p.B, blockIdx.x);
+        b = seq_of_token_warp(p.cu_q, p.B, blockIdx.x);
         g = blockIdx.x - __ldg(p.cu_q + b);
       }
     } else {
@@ -190,14 +207,25 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   {
     constexpr int CHUNKS_PER_ROW = C::DK / 8;
     uint8_t* qs = smem + C::OFF_Q;
-    for (int i = threadIdx.x; i < C::N * CHUNKS_PER_ROW; i += C::THREADS) {
-      const int n = i / CHUNKS_PER_ROW;
-      const int c = i % CHUNKS_PER_ROW;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      const int g = n / HI, j = n % HI;
-      if (g < nt && c * 8 < DIN)
-        v = *reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(t0 + g) * HI + j) * DIN + c * 8));
-      *reinterpret_cast<uint4*>(qs + (c / 8) * (C::N * 128) + sw128_offset(n, c % 8)) = v;
+    if constexpr (G == 1) {
+#pragma unroll
+      for (int u = 0; u < QPT; ++u) {
+        const int i = threadIdx.x + u * C::THREADS;
+        if (i < C::N * CHUNKS_PER_ROW) {
+          const int n = i / CHUNKS_PER_ROW, c = i % CHUNKS_PER_ROW;
+          *reinterpret_cast<uint4*>(qs + (c / 8) * (C::N * 128) + sw128_offset(n, c % 8)) = qreg[u];
+        }
+      }
+    } else {
+      for (int i = threadIdx.x; i < C::N * CHUNKS_PER_ROW; i += C::THREADS) {
+        const int n = i / CHUNKS_PER_ROW;
+        const int c = i % CHUNKS_PER_ROW;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        const int g = n / HI, j = n % HI;
+        if (g < nt && c * 8 < DIN)
+          v = *reinterpret_cast<const uint4*>(p.q + ((static_cast<int64_t>(t0 + g) * HI + j) * DIN + c * 8));
+        *reinterpret_cast<uint4*>(qs + (c / 8) * (C::N * 128) + sw128_offset(n, c % 8)) = v;
+      }
     }
     for (int i = threadIdx.x; i < G * HI; i += C::THREADS) {
       const int g = i / HI;

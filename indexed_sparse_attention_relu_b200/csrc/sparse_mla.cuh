@@ -171,16 +171,26 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     constexpr int ROUNDS = (CPR + 31) / 32;
     const int pw = warp - 4;
     const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * D;
-    // index of this lane's row (lanes 0..15), fetched one tile ahead
-    int nxt = (lane < 16 && k_begin + 16 * pw + lane < k_end) ? __ldg(idx_row + k_begin + 16 * pw + lane) : -1;
+    // index of this lane's row (lanes 0..15), fetched one tile ahead; the rows
+    // of the tile after next are prefetched into L2 (no shared memory needed),
+    // so the gather that fills a freed stage reads from L2
+    auto row_index = [&](int tile) -> int {
+      const int k = k_begin + tile * C::TK + 16 * pw + lane;
+      return (lane < 16 && tile < n_tiles && k < k_end) ? __ldg(idx_row + k) : -1;
+    };
+    auto prefetch_rows = [&](int s_row) {
+      if (s_row >= 0 && s_row < len) prefetch_l2(kv_seq + static_cast<int64_t>(s_row) * D, D * 2);
+    };
+    int nxt = row_index(0);
+    int nxt2 = row_index(1);
+    prefetch_rows(nxt);
+    prefetch_rows(nxt2);
     int issued = 0;
     for (int it = 0; it < n_tiles; ++it) {
       const int st = it & 1;
       const int cur = nxt;
-      if (it + 1 < n_tiles) {
-        const int kn = k_begin + (it + 1) * C::TK + 16 * pw + lane;
-        nxt = (lane < 16 && kn < k_end) ? __ldg(idx_row + kn) : -1;
-      }
+      nxt = nxt2;
+      nxt2 = row_index(it + 2);  // in flight during the stage wait and the gather
       if (!mbar_wait_warp(&kv_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
       const bool ok = cur >= 0 && cur < len;
       if (lane < 16 && cur != -1 && !ok) set_device_status(DSA_ERR_DEVICE_INDEX);
@@ -201,6 +211,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         }
       }
       cp_async_arrive_noinc(&kv_full[st]);
+      prefetch_rows(nxt2);
       ++issued;
     }
     cp_async_wait_all();  // nothing may still be landing when the CTA retires
