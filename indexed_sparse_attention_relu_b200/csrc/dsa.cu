@@ -12,6 +12,7 @@
 #include "indexer.cuh"
 #include "quant.cuh"
 #include "sparse_mla.cuh"
+#include "sparse_mla_pair.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -350,8 +351,70 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   return check_launch("sparse_mla");
 }
 
+// 128-head attention on 576-dim rows: CTA pairs split the row dims (see
+// sparse_mla_pair.cuh); key splits fill the SMs: one pair per (token, split),
+// at most 4 splits (cluster of 2 x splits CTAs).
+MlaPlan mla_pair_plan(int T, int K, int sms) {
+  const int tiles = (K + 63) / 64;
+  const int pairs = sms / 2;
+  int splits = T >= pairs ? 1 : pairs / T;
+  if (splits > PairCfg::MAX_SPLITS) splits = PairCfg::MAX_SPLITS;
+  if (splits > tiles) splits = tiles;
+  if (splits < 1) splits = 1;
+  const int tps = (tiles + splits - 1) / splits;
+  splits = (tiles + tps - 1) / tps;
+  return MlaPlan{splits, tps * 64};
+}
+
+dsa_status launch_mla_pair(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
+                           float* lse, cudaStream_t st, bool pdl) {
+  using C = PairCfg;
+  dsa_status s = set_smem(sparse_mla_pair_kernel, C::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  const int T = bt->num_q;
+  const MlaPlan pl = mla_pair_plan(T, k, num_sms());
+  MlaParams p;
+  p.cu_q = bt->cu_q;
+  p.seq_lens = bt->seq_lens;
+  p.B = bt->batch;
+  p.L_max = bt->max_seq_len;
+  p.T = T;
+  p.H = in->n_heads;
+  p.K = k;
+  p.idx = idx;
+  p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
+  p.keys_per_split = pl.keys_per_split;
+  p.splits = pl.splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pl.splits, T, 1);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 2 * pl.splits;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, sparse_mla_pair_kernel, static_cast<const __nv_bfloat16*>(in->q),
+                                           static_cast<const __nv_bfloat16*>(in->kv), p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla_pair launch: %s", cudaGetErrorString(e));
+  return check_launch("sparse_mla_pair");
+}
+
 dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
                       cudaStream_t st, bool pdl = false) {
+  if (in->d_latent == 512 && in->n_heads > 64) return launch_mla_pair(bt, in, idx, k, out, lse, st, pdl);
   const MlaPlan pl = mla_plan(bt->num_q, (in->n_heads + 63) / 64, k, num_sms());
   if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, st, pl, pdl);
   return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, st, pl, pdl);

@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     // so the gather that fills a freed stage reads from L2
     auto row_index = [&](int tile) -> int {
       const int k = k_begin + tile * C::TK + 16 * pw + lane;
-      return (lane < 16 && tile < n_tiles && k < k_end) ? __ldg(idx_row + k) : -1;
+      return (lane < 16 && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
     };
     auto prefetch_rows = [&](int s_row) {
       if (s_row >= 0 && s_row < len) prefetch_l2(kv_seq + static_cast<int64_t>(s_row) * D, D * 2);
@@ -284,14 +284,14 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     bool ok = true;
     uint8_t* p_tile = smem + C::OFF_P;
     // indices of the next tile (for the validity mask), one tile ahead
-    int i0n = (k_begin + lane < k_end) ? __ldg(idx_row + k_begin + lane) : -1;
-    int i1n = (k_begin + 32 + lane < k_end) ? __ldg(idx_row + k_begin + 32 + lane) : -1;
+    int i0n = (k_begin + lane < k_end) ? ld_dep(idx_row + k_begin + lane) : -1;
+    int i1n = (k_begin + 32 + lane < k_end) ? ld_dep(idx_row + k_begin + 32 + lane) : -1;
     for (int it = 0; it < n_tiles; ++it) {
       const int i0 = i0n, i1 = i1n;
       if (it + 1 < n_tiles) {
         const int kn = k_begin + (it + 1) * C::TK;
-        i0n = (kn + lane < k_end) ? __ldg(idx_row + kn + lane) : -1;
-        i1n = (kn + 32 + lane < k_end) ? __ldg(idx_row + kn + 32 + lane) : -1;
+        i0n = (kn + lane < k_end) ? ld_dep(idx_row + kn + lane) : -1;
+        i1n = (kn + 32 + lane < k_end) ? ld_dep(idx_row + kn + 32 + lane) : -1;
       }
       const unsigned v0 = __ballot_sync(0xffffffffu, i0 >= 0 && i0 < len);
       const unsigned v1 = __ballot_sync(0xffffffffu, i1 >= 0 && i1 < len);

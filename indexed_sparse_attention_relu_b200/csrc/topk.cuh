@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
 #pragma unroll
       for (int u = 0; u < BATCH; ++u) {
         const int i = base + u * THREADS + threadIdx.x;
-        v[u] = (i < n) ? __ldg(row + i) : 0.0f;
+        v[u] = (i < n) ? ld_dep(row + i) : 0.0f;
       }
 #pragma unroll
       for (int u = 0; u < BATCH; ++u) {
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
     }
     __syncthreads();
   }
-  auto key_at = [&](int i) -> uint32_t { return cached ? key_cache[i] : float_order_key(__ldg(row + i)); };
+  auto key_at = [&](int i) -> uint32_t { return cached ? key_cache[i] : float_order_key(ld_dep(row + i)); };
 
   uint32_t prefix = 0u, mask = 0u;
   int krem = p.K;
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_row_kernel(const TopkParams p
     if (vec && base + IPT <= n) {
 #pragma unroll
       for (int u = 0; u < IPT; u += 4) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(row + base + u));
+        const float4 f = ld_dep4(row + base + u);
         v[u] = f.x;
         v[u + 1] = f.y;
         v[u + 2] = f.z;
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(THREADS, 1) topk_row_kernel(const TopkParams p
       }
     } else {
 #pragma unroll
-      for (int u = 0; u < IPT; ++u) v[u] = (base + u < n) ? __ldg(row + base + u) : 0.0f;
+      for (int u = 0; u < IPT; ++u) v[u] = (base + u < n) ? ld_dep(row + base + u) : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < IPT; u += 4) {
