@@ -161,10 +161,14 @@ dsa_status dsa_topk(const dsa_batch *batch, const float *scores, int64_t score_l
  * out: bf16 [T, n_heads, d_latent]:  sum_i softmax_i(scale * q.kv_i) * kv_i[0:d_latent]
  * lse: fp32 [T, n_heads] natural-log sum-exp of the scaled logits, or NULL.
  * A row with no valid index gets out = 0 and lse = -inf.
- * ws: unused (dsa_workspace_size(DSA_OP_SPARSE_MLA, ...) is 0); may be NULL.
- * Work split: one CTA per (query, 64-head block, key split); the key splits
- * of a query form a thread-block cluster and merge through distributed
- * shared memory, so no intermediate goes to global memory. */
+ * ws: at least dsa_workspace_size(DSA_OP_SPARSE_MLA, ...) bytes, 16-byte
+ *   aligned (the size is 0, and ws may be NULL, when the batch has enough
+ *   queries to fill the GPU without splitting their keys).
+ * Work split: one CTA per (query, 64-head block, key split). The key splits
+ * of a query form a thread-block cluster; each leaves its unnormalised
+ * output rows and (max, sum) statistics in ws and, after the cluster
+ * barrier, the split that owns a head merges it. DSA_ERR_WORKSPACE_TOO_SMALL
+ * if ws is smaller than that call needs. */
 dsa_status dsa_sparse_mla_attn(const dsa_batch *batch, const dsa_mla_in *in, const int32_t *idx,
                                int32_t k, void *out, float *lse, void *ws, size_t ws_bytes,
                                dsa_stream_t stream);

@@ -12,7 +12,6 @@
 #include "indexer.cuh"
 #include "quant.cuh"
 #include "sparse_mla.cuh"
-#include "sparse_mla_pair.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -174,8 +173,28 @@ MlaPlan mla_plan(int T, int HB, int K, int sms) {
   return MlaPlan{splits, tps * 64};
 }
 
-// The attention needs no workspace: split partials merge inside a cluster.
-size_t mla_ws_bytes() { return 0; }
+// Workspace of the attention: with key splits, every split CTA leaves its
+// unnormalised O rows (64 x d_latent fp32) and per-row (max, sum) in global
+// memory for the merge. Sized for the largest supported latent dim.
+constexpr int kMlaMaxLatent = 512;
+
+size_t mla_part_bytes(int T, int hb, int splits, int dc) {
+  if (splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(T) * hb * splits * 64;
+  return align256(rows * dc * sizeof(float)) + align256(rows * sizeof(float2));
+}
+
+// Upper bound over the head-block counts a call can use (1 or 2).
+size_t mla_ws_bytes(const dsa_batch* bt, int k) {
+  const int T = bt->num_q;
+  size_t need = 0;
+  for (int hb = 1; hb <= 2; ++hb) {
+    const MlaPlan pl = mla_plan(T, hb, k, num_sms());
+    const size_t b = mla_part_bytes(T, hb, pl.splits, kMlaMaxLatent);
+    need = b > need ? b : need;
+  }
+  return need;
+}
 
 // ---------------------------------------------------------------- launches
 template <typename Kern>
@@ -301,7 +320,7 @@ dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int
 
 template <int D, int DC>
 dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
-                        float* lse, cudaStream_t st, const MlaPlan& pl, bool pdl) {
+                        float* lse, void* ws, size_t ws_bytes, cudaStream_t st, const MlaPlan& pl, bool pdl) {
   using C = MlaCfg<D, DC>;
   auto kern = sparse_mla_kernel<D, DC>;
   dsa_status s = set_smem(kern, C::SMEM_BYTES);
@@ -324,6 +343,17 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   const int hb = (H + 63) / 64;
+  p.part_o = nullptr;
+  p.part_ml = nullptr;
+  if (pl.splits > 1) {
+    const size_t need = mla_part_bytes(T, hb, pl.splits, DC);
+    if (!ws || ws_bytes < need)
+      return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "attention workspace %zu < %zu bytes", ws_bytes, need);
+    if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    const size_t rows = static_cast<size_t>(T) * hb * pl.splits * 64;
+    p.part_o = static_cast<float*>(ws);
+    p.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(ws) + align256(rows * DC * sizeof(float)));
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(T, hb, pl.splits);
   cfg.blockDim = dim3(C::THREADS);
@@ -351,73 +381,11 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   return check_launch("sparse_mla");
 }
 
-// 128-head attention on 576-dim rows: CTA pairs split the row dims (see
-// sparse_mla_pair.cuh); key splits fill the SMs: one pair per (token, split),
-// at most 4 splits (cluster of 2 x splits CTAs).
-MlaPlan mla_pair_plan(int T, int K, int sms) {
-  const int tiles = (K + 63) / 64;
-  const int pairs = sms / 2;
-  int splits = T >= pairs ? 1 : pairs / T;
-  if (splits > PairCfg::MAX_SPLITS) splits = PairCfg::MAX_SPLITS;
-  if (splits > tiles) splits = tiles;
-  if (splits < 1) splits = 1;
-  const int tps = (tiles + splits - 1) / splits;
-  splits = (tiles + tps - 1) / tps;
-  return MlaPlan{splits, tps * 64};
-}
-
-dsa_status launch_mla_pair(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
-                           float* lse, cudaStream_t st, bool pdl) {
-  using C = PairCfg;
-  dsa_status s = set_smem(sparse_mla_pair_kernel, C::SMEM_BYTES);
-  if (s != DSA_OK) return s;
-  const int T = bt->num_q;
-  const MlaPlan pl = mla_pair_plan(T, k, num_sms());
-  MlaParams p;
-  p.cu_q = bt->cu_q;
-  p.seq_lens = bt->seq_lens;
-  p.B = bt->batch;
-  p.L_max = bt->max_seq_len;
-  p.T = T;
-  p.H = in->n_heads;
-  p.K = k;
-  p.idx = idx;
-  p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
-  p.keys_per_split = pl.keys_per_split;
-  p.splits = pl.splits;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pl.splits, T, 1);
-  cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  int na = 0;
-  attr[na].id = cudaLaunchAttributeClusterDimension;
-  attr[na].val.clusterDim.x = 2 * pl.splits;
-  attr[na].val.clusterDim.y = 1;
-  attr[na].val.clusterDim.z = 1;
-  ++na;
-  if (pdl) {
-    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[na].val.programmaticStreamSerializationAllowed = 1;
-    ++na;
-  }
-  cfg.attrs = attr;
-  cfg.numAttrs = na;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, sparse_mla_pair_kernel, static_cast<const __nv_bfloat16*>(in->q),
-                                           static_cast<const __nv_bfloat16*>(in->kv), p);
-  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla_pair launch: %s", cudaGetErrorString(e));
-  return check_launch("sparse_mla_pair");
-}
-
 dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
-                      cudaStream_t st, bool pdl = false) {
-  if (in->d_latent == 512 && in->n_heads > 64) return launch_mla_pair(bt, in, idx, k, out, lse, st, pdl);
+                      void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false) {
   const MlaPlan pl = mla_plan(bt->num_q, (in->n_heads + 63) / 64, k, num_sms());
-  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, st, pl, pdl);
-  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, st, pl, pdl);
+  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
+  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
 }
 
 }  // namespace
@@ -455,10 +423,10 @@ size_t dsa_workspace_size(int op, const dsa_batch* batch, int32_t k, int32_t h_i
     case DSA_OP_TOPK:
       return 0;
     case DSA_OP_SPARSE_MLA:
-      return mla_ws_bytes();
+      return mla_ws_bytes(batch, k);
     case DSA_OP_FUSED_DECODE:
       return align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float)) +
-             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes();
+             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes(batch, k);
     default:
       return 0;
   }
@@ -498,10 +466,8 @@ dsa_status dsa_sparse_mla_attn(const dsa_batch* batch, const dsa_mla_in* in, con
   if (!idx || !out) return fail(DSA_ERR_INVALID_ARGUMENT, "idx and out must be non-NULL");
   if (!aligned16(out) || !aligned16(idx)) return fail(DSA_ERR_MISALIGNED, "idx and out must be 16-byte aligned");
   if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
-  (void)ws;
-  (void)ws_bytes;
   if (batch->num_q == 0) return DSA_OK;
-  return launch_mla(batch, in, idx, k, out, lse, reinterpret_cast<cudaStream_t>(stream));
+  return launch_mla(batch, in, idx, k, out, lse, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in, const dsa_mla_in* mla_in,
@@ -519,7 +485,8 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
   const int T = batch->num_q;
   const size_t sc_bytes = align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float));
   const size_t id_bytes = align256(static_cast<size_t>(T) * k * sizeof(int32_t));
-  const size_t need = sc_bytes + id_bytes + mla_ws_bytes();
+  const size_t mla_bytes = mla_ws_bytes(batch, k);
+  const size_t need = sc_bytes + id_bytes + mla_bytes;
   if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
   if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -539,7 +506,9 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
   const bool pdl = stage_events == nullptr;
   if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st, pdl)) != DSA_OK) return s;
   if ((s = rec(2)) != DSA_OK) return s;
-  if ((s = launch_mla(batch, mla_in, idx, k, out, lse, st, pdl)) != DSA_OK) return s;
+  if ((s = launch_mla(batch, mla_in, idx, k, out, lse, static_cast<uint8_t*>(ws) + sc_bytes + id_bytes, mla_bytes, st,
+                      pdl)) != DSA_OK)
+    return s;
   return rec(3);
 }
 
@@ -657,8 +626,8 @@ dsa_status noalloc_scratch(void** out) {
 dsa_status launch_mla_unsplit(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
                               float* lse, cudaStream_t st) {
   const MlaPlan pl{1, ((k + 63) / 64) * 64};
-  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, st, pl, false);
-  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, st, pl, false);
+  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false);
+  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false);
 }
 
 }  // namespace

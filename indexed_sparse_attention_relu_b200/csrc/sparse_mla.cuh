@@ -8,32 +8,36 @@
 //   out[t,h,:] = sum_i softmax(z)_i * kv[b,s_i,0:d_c]     (value = latent part)
 //   lse[t,h] = log sum_i exp(z_i)
 //
-// One CTA = (token, 64-head block, key split); the key splits of one
-// (token, head block) form a thread-block cluster. Per tile of 64 selected keys:
-//  * four producer warps gather the 64 rows with 16-byte cp.async straight
-//    into the 128-byte-swizzled K-major layout (one warp instruction moves
-//    512 contiguous bytes of a row, three cover a 1152-byte row); each thread
-//    signals its copies through an asynchronous mbarrier arrival, so the
-//    producers run one tile ahead without blocking; an index of -1 or out of
-//    range zero-fills its row (two-stage ring);
+// One CTA = (token, 64-head block, key split). Each CTA gathers whole rows
+// (a gather costs the issuing warps per row, not per byte, so whole rows are
+// the cheapest unit). Per tile of 64 selected keys:
+//  * eight producer warps gather the 64 rows with 16-byte cp.async straight
+//    into the 128-byte-swizzled K-major layout; the 16-byte chunks of a warp's
+//    eight rows are packed 32 to an instruction (512 contiguous bytes), and
+//    every thread signals its copies through an asynchronous mbarrier
+//    arrival; an index of -1 or out of range zero-fills its row (three-stage
+//    ring);
 //  * one thread issues S = Q K^T (M = 64 heads, N = 64 keys, K = D) and
 //    O += P V (M = 64, N = d_c in 256-wide pieces, K = 64 keys) on tcgen05;
 //    the value operand is the same shared-memory tile read as an MN-major
 //    matrix, so each row is gathered once;
-//  * with M = 64 an accumulator uses lanes 0-15 of each TMEM sub-partition,
-//    so O (all d_c columns) sits at lane offset 0 and S at lane offset 16 of
-//    the same columns: both fit in one SM's TMEM;
-//  * 4 softmax warps read S with 16-lane TMEM loads, so all 32 threads work:
-//    thread t holds head rows t/4 and t/4 + 8 of its warp's 16 and 16 of the
-//    64 keys; they run an online softmax in the exp2 domain with lazy
-//    rescaling: O is only rescaled (TMEM load/scale/store) when a row maximum
-//    grows by more than 2^8, which keeps P <= 256 and the result exact;
+//  * with M = 64 an accumulator uses lanes 0-15 of each TMEM sub-partition:
+//    O (all d_c columns) sits at lane offset 0; S (64 columns) and Q (the A
+//    operand of S = Q K^T, D/2 columns of bf16 pairs) sit at lane offset 16.
+//    Q arrives by TMA in the third gather stage, which is handed to the
+//    gather once the softmax warps have moved Q into tensor memory;
+//  * 4 softmax warps read S with 16-lane TMEM loads (thread t holds head rows
+//    t/4 and t/4 + 8 of its warp's 16 and 16 of the 64 keys) and run an
+//    online softmax in the exp2 domain with lazy rescaling: O is only
+//    rescaled (16-lane TMEM load/scale/store) when a row maximum grows by
+//    more than 2^8, which keeps P <= 256 and the result exact;
 //  * P is written as bf16 to shared memory (A operand of the PV product).
-// The split partials (O, running max, running sum) are merged inside the
-// cluster: every CTA sends each head row to the CTA that owns that head
-// (owner = head mod splits) through distributed shared memory, and the owner
-// writes the bf16 output and the lse. All cross-CTA handshakes are mbarriers
-// with bounded waits.
+// Key splits of one (token, head block) form a thread-block cluster: every
+// CTA writes its unnormalised O rows and (running max, running sum) to the
+// workspace in global memory, the cluster barrier orders those writes, and
+// head h is then finalised by the CTA of split h mod splits (distributed
+// shared memory is far slower than L2 for bulk data, so it carries none).
+// Every wait is bounded.
 #pragma once
 #include "dsa_common.cuh"
 
@@ -53,66 +57,121 @@ struct MlaParams {
   int32_t splits;            // == cluster size along z
   __nv_bfloat16* out;        // [T, H, DC]
   float* lse;                // [T, H] or null
+  float* part_o;             // [T, HB, splits][DC / 4][64][4] split partials (splits > 1)
+  float2* part_ml;           // [T, HB, splits, 64] (running max, running sum)
 };
 
 template <int D, int DC>
 struct MlaCfg {
-  static constexpr int DP = ((D + 63) / 64) * 64;   // K extent of the QK^T product (whole atoms)
+  static constexpr int DP = ((D + 63) / 64) * 64;   // K extent of the stored rows (whole atoms)
   static constexpr int AKQ = DP / 64;               // 128-byte atom columns per row
   static constexpr int HB = 64;                     // heads per CTA (MMA M)
   static constexpr int TK = 64;                     // keys per tile (QK^T N, PV K)
+  static constexpr int KSTEPS = (D + 15) / 16;      // K steps of QK^T
   static constexpr int ATOM_COL = 64 * 128;         // bytes of one atom column of a 64-row tile
-  static constexpr int Q_BYTES = HB * DP * 2;
   static constexpr int KV_BYTES = TK * DP * 2;
+  static constexpr int Q_BYTES = HB * DP * 2;       // staged in the last gather stage
   static constexpr int P_BYTES = HB * TK * 2;
-  static constexpr int NST = 2;
+  static constexpr int NST = 3;
   static constexpr int N_PV = DC < 256 ? DC : 256;
   static constexpr int PV_MMAS = DC / N_PV;
-  static constexpr int TMEM_COLS = DC <= 32 ? 32 : DC <= 64 ? 64 : DC <= 128 ? 128 : DC <= 256 ? 256 : 512;
-  static constexpr int NUM_WARPS = 9;  // 0-3 softmax/epilogue, 4-7 gather producers, 8 MMA + TMEM owner
+  static constexpr uint32_t COL_S = 0;              // lane offset 16
+  static constexpr uint32_t COL_Q = 64;             // lane offset 16, DP/2 columns
+  static constexpr int TMEM_NEED = (DC > (int)COL_Q + DP / 2) ? DC : (int)COL_Q + DP / 2;
+  static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
+  static constexpr int PRODUCERS = 8;               // gather warps
+  static constexpr int NUM_WARPS = 4 + PRODUCERS + 1;  // 0-3 softmax/epilogue, 4-11 gather, 12 MMA + TMEM owner
   static constexpr int THREADS = NUM_WARPS * 32;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + Q_BYTES;
+  static constexpr int OFF_KV = 0;
   static constexpr int OFF_P = OFF_KV + NST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_P + P_BYTES;
   static constexpr int NUM_BARS = 2 * NST + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int MAX_SPLITS = 8;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(64, TK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(64, N_PV, false, true);
   static_assert(DC % N_PV == 0 && DC % 64 == 0, "latent dim must be a multiple of 64");
+  static_assert(TMEM_NEED <= 512, "TMEM budget");
+  static_assert(Q_BYTES <= KV_BYTES, "Q is staged in one gather stage");
+  static_assert((DP / 2) % 32 == 0, "Q columns come in 32-column groups");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  // merge buffers reuse the KV ring (partial O rows) and the P tile (statistics);
-  // S * ceil(64 / S) entries, at most 70 (S = 7) for S <= 8
-  static_assert(70 * DC * 4 <= NST * KV_BYTES, "merge buffer must fit in the KV ring");
-  static_assert(70 * 8 <= P_BYTES, "merge statistics must fit in the P tile");
 };
+
+// 16 lanes x 256 bits, 8 repetitions (64 columns): the store counterpart of
+// tmem_ld16x256_x8 (same register layout).
+__device__ __forceinline__ void tmem_st16x256_x8(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
+// 16 lanes x 256 bits, 4 repetitions (32 columns), store.
+__device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ uint2 ld_shared_v2u(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
+  return v;
+}
+
+// Packed bf16 pairs of Q for TMEM column `col` (dims 2col, 2col+1) of the
+// thread's two head rows, read from the TMA-staged swizzled Q tile.
+template <int ATOM_COL>
+__device__ __forceinline__ void q_pair(uint32_t q_stage, int ha, int hbr, int col, uint32_t& xa0, uint32_t& xa1,
+                                       uint32_t& xb0, uint32_t& xb1) {
+  const int d = 2 * col;                                        // first dim of the two columns
+  const uint32_t off = (d >> 6) * ATOM_COL + (d & 7) * 2;       // atom column, byte in the chunk
+  const uint2 x = ld_shared_v2u(q_stage + off + sw128_offset(ha, (d & 63) >> 3));
+  const uint2 y = ld_shared_v2u(q_stage + off + sw128_offset(hbr, (d & 63) >> 3));
+  xa0 = x.x;
+  xa1 = x.y;
+  xb0 = y.x;
+  xb1 = y.y;
+}
 
 template <int D, int DC>
 __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     sparse_mla_kernel(const __nv_bfloat16* __restrict__ kv, const __grid_constant__ CUtensorMap qmap,
                       const MlaParams p) {
   using C = MlaCfg<D, DC>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The swizzled tiles need 1024-byte alignment; the dynamic window starts at
+  // the same offset in every CTA, so either all CTAs leave here or none.
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) set_device_status(DSA_ERR_DEVICE_LAYOUT);
+    return;
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;             // [NST] gather producers -> MMA
   uint64_t* kv_empty = bars + C::NST;   // [NST] MMA (PV done) -> gather producers
-  uint64_t* q_full = kv_empty + C::NST; // TMA -> MMA
-  uint64_t* s_full = q_full + 1;        // MMA (S ready) -> softmax
+  uint64_t* q_full = kv_empty + C::NST; // TMA (Q staged) -> softmax warps
+  uint64_t* q_moved = q_full + 1;       // softmax warps (Q in TMEM) -> MMA, and the last stage -> gather
+  uint64_t* s_full = q_moved + 1;       // MMA (S ready) -> softmax
   uint64_t* s_empty = s_full + 1;       // softmax (S read) -> MMA
   uint64_t* p_full = s_empty + 1;       // softmax (P written) -> MMA
   uint64_t* o_done = p_full + 1;        // MMA (PV done) -> softmax
   uint64_t* drain = o_done + 1;
-  uint64_t* ready = drain + 1;          // merge: every CTA of the cluster has finished its loop
-  uint64_t* recv = ready + 1;           // merge: every partial row destined here has arrived
-  int32_t* misc = reinterpret_cast<int32_t*>(smem + C::OFF_MISC);
-  // misc: [0] TMEM base, [1] abort
+  int32_t* misc = reinterpret_cast<int32_t*>(smem + C::OFF_MISC);  // [0] TMEM base, [1] abort
   volatile int* abort_flag = misc + 1;
 
   const int t = blockIdx.x;
-  const int h0 = blockIdx.y * C::HB;
+  const int hb = blockIdx.y;
+  const int h0 = hb * C::HB;
   const int split = blockIdx.z;
   const int S = p.splits;
   const int warp = warp_id();
@@ -123,126 +182,103 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
   const int k_end = min(p.K, k_begin + p.keys_per_split);
   const int n_tiles = (k_end - k_begin + C::TK - 1) / C::TK;  // >= 1 by construction
   const int32_t* idx_row = p.idx + static_cast<int64_t>(t) * p.K;
+  const uint32_t q_stage = smem_u32(smem + C::OFF_KV + (C::NST - 1) * C::KV_BYTES);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
-      mbar_init(&kv_full[i], 128);  // one asynchronous arrival per producer thread
+      mbar_init(&kv_full[i], C::PRODUCERS * 32);  // one asynchronous arrival per producer thread
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(q_full, 1);
+    mbar_init(q_moved, 4);
     mbar_init(s_full, 1);
     mbar_init(s_empty, 4);
     mbar_init(p_full, 4);
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
-    mbar_init(ready, S);
-    mbar_init(recv, 64 * S);
     misc[1] = 0;
     fence_mbar_init();
     prefetch_tensormap(&qmap);
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(reinterpret_cast<uint32_t*>(misc), C::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
-  if (S > 1)
-    cluster_sync_all();  // peers' barriers are initialised before any remote arrive
-  else
-    __syncthreads();
+  __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = static_cast<uint32_t>(misc[0]);
-  const uint32_t tmem_s = tmem_base + (16u << 16);  // S at lane offset 16 (M = 64 layout)
+  const uint32_t lo16 = 16u << 16;  // lane offset 16: S and Q (M = 64 layout)
 
-  if (warp == 8 && lane == 0) {
+  if (warp == 12 && lane == 0) {
     // the query block is an input of the call, not of the Top-K: load it now
     mbar_arrive_expect_tx(q_full, C::Q_BYTES);
-    const uint32_t qs = smem_u32(smem + C::OFF_Q);
 #pragma unroll
-    for (int c = 0; c < C::AKQ; ++c) tma_load_2d(qs + c * C::ATOM_COL, &qmap, c * 64, t * p.H + h0, q_full);
+    for (int c = 0; c < C::AKQ; ++c) tma_load_2d(q_stage + c * C::ATOM_COL, &qmap, c * 64, t * p.H + h0, q_full);
   }
-  pdl_wait_prior();  // the selected indices (Top-K output) are complete from here on
 
-  if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ gather producers (4 warps)
-    // warp pw copies rows 16pw .. 16pw+15 of each 64-key tile; for one row the
-    // whole warp issues 16-byte chunks 32 at a time (512 contiguous bytes)
-    constexpr int CPR = C::DP / 8;                // 16-byte chunks per padded row
-    constexpr int ROUNDS = (CPR + 31) / 32;
+  if (warp >= 4 && warp < 12) {
+    // ------------------------------------------------------------ gather producers (8 warps)
+    // Warp pw copies rows 8 pw .. 8 pw + 7 of each tile. Their 16-byte chunks
+    // are numbered row-major (CPR per row) and issued 32 per instruction, so
+    // most instructions move 512 contiguous bytes of one row.
+    pdl_wait_prior();
+    constexpr int CPR = C::DP / 8;                 // 16-byte chunks per stored row
+    constexpr int ROUNDS = (8 * CPR + 31) / 32;    // instructions per warp per tile
     const int pw = warp - 4;
     const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * D;
-    // index of this lane's row (lanes 0..15), fetched one tile ahead; the rows
-    // of the tile after next are prefetched into L2 (no shared memory needed),
-    // so the gather that fills a freed stage reads from L2
     auto row_index = [&](int tile) -> int {
-      const int k = k_begin + tile * C::TK + 16 * pw + lane;
-      return (lane < 16 && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
-    };
-    auto prefetch_rows = [&](int s_row) {
-      if (s_row >= 0 && s_row < len) prefetch_l2(kv_seq + static_cast<int64_t>(s_row) * D, D * 2);
+      const int k = k_begin + tile * C::TK + 8 * pw + lane;
+      return (lane < 8 && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
     };
     int nxt = row_index(0);
-    int nxt2 = row_index(1);
-    prefetch_rows(nxt);
-    prefetch_rows(nxt2);
-    int issued = 0;
-    for (int it = 0; it < n_tiles; ++it) {
-      const int st = it & 1;
+    bool ok = true;
+    for (int it = 0; it < n_tiles && ok; ++it) {
+      const int sl = it % C::NST;
+      const uint32_t use = static_cast<uint32_t>(it / C::NST);
       const int cur = nxt;
-      nxt = nxt2;
-      nxt2 = row_index(it + 2);  // in flight during the stage wait and the gather
-      if (!mbar_wait_warp(&kv_empty[st], ((it >> 1) & 1) ^ 1, abort_flag)) break;
-      const bool ok = cur >= 0 && cur < len;
-      if (lane < 16 && cur != -1 && !ok) set_device_status(DSA_ERR_DEVICE_INDEX);
-      const uint32_t stage = smem_u32(smem + C::OFF_KV + st * C::KV_BYTES);
-#pragma unroll 4
-      for (int rr = 0; rr < 16; ++rr) {
-        const int r = 16 * pw + rr;                         // key slot in the tile
-        const int srow = __shfl_sync(0xffffffffu, ok ? cur : -1, rr);
-        const __nv_bfloat16* src_row = kv_seq + static_cast<int64_t>(srow < 0 ? 0 : srow) * D;
-#pragma unroll
-        for (int q = 0; q < ROUNDS; ++q) {
-          const int c = 32 * q + lane;                      // 16-byte chunk of the row
-          if (c < CPR) {
-            const bool has = srow >= 0 && c * 8 < D;
-            cp_async_16(stage + (c / 8) * C::ATOM_COL + sw128_offset(r, c % 8), has ? src_row + c * 8 : kv,
-                        has ? 16u : 0u);
-          }
+      nxt = row_index(it + 1);  // in flight during the stage wait and the copies
+      // the last stage holds Q until the softmax warps have moved it to TMEM
+      if (it == C::NST - 1) ok = mbar_wait_warp(q_moved, 0, abort_flag);
+      if (ok) ok = mbar_wait_warp(&kv_empty[sl], (use & 1u) ^ 1u, abort_flag);
+      if (!ok) break;
+      const bool okr = cur >= 0 && cur < len;
+      if (lane < 8 && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
+      const int mine = okr ? cur : -1;
+      const uint32_t stage = smem_u32(smem + C::OFF_KV + sl * C::KV_BYTES);
+#pragma unroll 2
+      for (int q = 0; q < ROUNDS; ++q) {
+        const int flat = q * 32 + lane;                  // chunk number within the warp's rows
+        const int rl = flat / CPR;                       // row of the warp (0..7)
+        const int c = flat - rl * CPR;                   // 16-byte chunk of the row
+        const int srow = __shfl_sync(0xffffffffu, mine, rl & 7);
+        if (flat < 8 * CPR) {
+          const int r = 8 * pw + rl;
+          const bool has = srow >= 0 && c * 8 < D;
+          const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * D + (has ? c * 8 : 0);
+          cp_async_16(stage + (c >> 3) * C::ATOM_COL + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
         }
       }
-      cp_async_arrive_noinc(&kv_full[st]);
-      prefetch_rows(nxt2);
-      ++issued;
+      cp_async_arrive_noinc(&kv_full[sl]);
     }
     cp_async_wait_all();  // nothing may still be landing when the CTA retires
-    (void)issued;
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t q_base = smem_u32(smem + C::OFF_Q);
       const uint32_t p_base = smem_u32(smem + C::OFF_P);
+      const uint32_t tmem_s = tmem_base + lo16 + C::COL_S;
+      const uint32_t tmem_q = tmem_base + lo16 + C::COL_Q;
       auto issue_s = [&](int it) {
-        const uint32_t kvb = smem_u32(smem + C::OFF_KV + (it & 1) * C::KV_BYTES);
+        const uint32_t kvb = smem_u32(smem + C::OFF_KV + (it % C::NST) * C::KV_BYTES);
 #pragma unroll
-        for (int k = 0; k < C::DP / 16; ++k) {
-          const uint64_t a = smem_desc_sw128(q_base + (k / 4) * C::ATOM_COL + (k % 4) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(kvb + (k / 4) * C::ATOM_COL + (k % 4) * 32, 16, 1024);
-          umma_f16(tmem_s, a, bd, C::IDESC_S, k > 0 ? 1u : 0u);
+        for (int k = 0; k < C::KSTEPS; ++k) {
+          const uint64_t bd = smem_desc_sw128(kvb + (k >> 2) * C::ATOM_COL + (k & 3) * 32, 16, 1024);
+          umma_f16_ts(tmem_s, tmem_q + 8 * k, bd, C::IDESC_S, k > 0 ? 1u : 0u);
         }
         umma_commit(s_full);
       };
-      // Order: S(0), then per tile PV(it) followed by S(it+1). The gather of
-      // tile it+1 only waits for PV(it-1), which is issued before S(it+1).
-      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
-      if (ok) {
-        fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor core reads
-        tc_fence_after();
-        issue_s(0);
-      }
-      for (int it = 0; ok && it < n_tiles; ++it) {
-        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t kvb = smem_u32(smem + C::OFF_KV + (it & 1) * C::KV_BYTES);
+      auto issue_pv = [&](int it) {
+        const uint32_t kvb = smem_u32(smem + C::OFF_KV + (it % C::NST) * C::KV_BYTES);
 #pragma unroll
         for (int nb = 0; nb < C::PV_MMAS; ++nb) {
 #pragma unroll
@@ -255,38 +291,91 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
             umma_f16(tmem_base + nb * C::N_PV, a, bd, C::IDESC_PV, (it > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        umma_commit(&kv_empty[it & 1]);
+        umma_commit(&kv_empty[it % C::NST]);
         umma_commit(o_done);
-        if (it + 1 < n_tiles) {
-          if (!(ok = mbar_wait(s_empty, it & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(&kv_full[(it + 1) & 1], ((it + 1) >> 1) & 1, abort_flag))) break;
-          fence_proxy_async_smem();
+      };
+      bool ok = mbar_wait(q_moved, 0, abort_flag);
+      int s_next = 0, pv_next = 0;
+      uint64_t t0 = globaltimer();
+      // Issue whichever product is ready (non-blocking tests, so one barrier
+      // never holds up another): S(j) needs tile j gathered and the softmax
+      // done reading S(j-1) (one S buffer); PV(j) needs P(j).
+      while (ok && pv_next < n_tiles) {
+        bool progressed = false;
+        if (s_next < n_tiles && (s_next == 0 || mbar_test(smem_u32(s_empty), (s_next - 1) & 1)) &&
+            mbar_test(smem_u32(&kv_full[s_next % C::NST]), (s_next / C::NST) & 1)) {
+          fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor core reads
           tc_fence_after();
-          issue_s(it + 1);
+          issue_s(s_next);
+          ++s_next;
+          progressed = true;
+        }
+        if (pv_next < s_next && mbar_test(smem_u32(p_full), pv_next & 1)) {
+          tc_fence_after();
+          issue_pv(pv_next);
+          ++pv_next;
+          progressed = true;
+        }
+        if (progressed) {
+          t0 = globaltimer();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (globaltimer() - t0 > kWaitLimitNs) {
+          set_device_status(DSA_ERR_DEVICE_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
         }
       }
       umma_commit(drain);
       volatile int never = 0;
       mbar_wait(drain, 0, &never);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue (warps 0..3)
     const int sw = warp;                                   // TMEM sub-partition
     const uint32_t lane_addr = static_cast<uint32_t>(sw * 32) << 16;
-    const bool is_s = lane >= 16;                          // threads 16..31 own S rows
-    const int h_local = sw * 16 + (lane & 15);             // head row inside the block
-    // Rows of S this thread handles in the 16-lane layout: head rows ra, ra+8
-    // of the warp's 16 (h_local = sw*16 + row) and key columns 8j + cc, +1.
+    // Rows this thread handles in the 16-lane layout: head rows ra, ra+8 of
+    // the warp's 16 (h_local = sw*16 + row) and columns 8j + cc, +1.
     const int ra = lane >> 2;
     const int cc = 2 * (lane & 3);
+    bool ok = mbar_wait_warp(q_full, 0, abort_flag);
+    if (ok) {
+      // Q -> TMEM (lanes 16..31 of this sub-partition, column COL_Q + c holds
+      // dims 2c, 2c+1), in the 16x256b layout of rows ra, ra+8
+      const int ha = sw * 16 + ra, hbr = ha + 8;
+      constexpr int QCOLS = C::DP / 2;
+#pragma unroll
+      for (int g = 0; g < QCOLS / 64; ++g) {
+        uint32_t v[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          q_pair<C::ATOM_COL>(q_stage, ha, hbr, 64 * g + 8 * j + cc, v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                              v[4 * j + 3]);
+        tmem_st16x256_x8(tmem_base + lane_addr + lo16 + C::COL_Q + 64 * g, v);
+      }
+      if constexpr (QCOLS % 64 == 32) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          q_pair<C::ATOM_COL>(q_stage, ha, hbr, (QCOLS / 64) * 64 + 8 * j + cc, v[4 * j], v[4 * j + 1],
+                              v[4 * j + 2], v[4 * j + 3]);
+        tmem_st16x256_x4(tmem_base + lane_addr + lo16 + C::COL_Q + (QCOLS / 64) * 64, v);
+      }
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(q_moved);  // also on failure: every wait stays bounded
+    pdl_wait_prior();  // the selected indices (Top-K output) are complete from here on
+
     float m_a = -INFINITY, m_b = -INFINITY;  // running max per row (log2 domain)
     float l_a = 0.0f, l_b = 0.0f;            // this thread's share of the running sums
-    bool ok = true;
     uint8_t* p_tile = smem + C::OFF_P;
     // indices of the next tile (for the validity mask), one tile ahead
     int i0n = (k_begin + lane < k_end) ? ld_dep(idx_row + k_begin + lane) : -1;
     int i1n = (k_begin + 32 + lane < k_end) ? ld_dep(idx_row + k_begin + 32 + lane) : -1;
-    for (int it = 0; it < n_tiles; ++it) {
+    for (int it = 0; it < n_tiles && ok; ++it) {
       const int i0 = i0n, i1 = i1n;
       if (it + 1 < n_tiles) {
         const int kn = k_begin + (it + 1) * C::TK;
@@ -298,8 +387,12 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
       if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
       float v[32];
-      tmem_ld16x256_x8(tmem_s + lane_addr, v);
+      tmem_ld16x256_x8(tmem_base + lane_addr + lo16 + C::COL_S, v);
       tmem_wait_ld();
+      // the S buffer is free again: the next QK^T may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_empty);
       // v[4j + 0/1] = row ra, cols 8j+cc, +1; v[4j + 2/3] = row ra+8, same cols
       float ta = -INFINITY, tb = -INFINITY;
 #pragma unroll
@@ -333,30 +426,28 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
       }
       bool o_waited = false;
       if (__any_sync(0xffffffffu, (need_a || need_b) && it > 0)) {
-        // O already holds earlier tiles: wait for PV(it-1), then rescale those rows
+        // O already holds earlier tiles: wait for PV(it-1), then rescale
+        // rows ra, ra+8 (16-lane accesses touch O's lanes only)
         if (!(ok = mbar_wait_warp(o_done, (it - 1) & 1, abort_flag))) break;
         o_waited = true;
         tc_fence_after();
-        // O row r (lanes 0..15 in the 32-lane layout) is row ra of thread 4(r%8) (a if r < 8, else b)
-        const int src = 4 * (lane & 7);
-        const float ga = __shfl_sync(0xffffffffu, fa, src);
-        const float gb = __shfl_sync(0xffffffffu, fb, src);
-        const float fo = (lane < 8) ? ga : gb;
-        for (int c = 0; c < DC; c += 16) {
-          float o[16];
-          tmem_ld16(tmem_base + lane_addr + c, o);
+#pragma unroll 1
+        for (int c = 0; c < DC; c += 64) {
+          float o[32];
+          tmem_ld16x256_x8(tmem_base + lane_addr + c, o);
           tmem_wait_ld();
-          if (lane < 16) {
+          uint32_t w[32];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) o[u] *= fo;
+          for (int j = 0; j < 8; ++j) {
+            w[4 * j + 0] = __float_as_uint(o[4 * j + 0] * fa);
+            w[4 * j + 1] = __float_as_uint(o[4 * j + 1] * fa);
+            w[4 * j + 2] = __float_as_uint(o[4 * j + 2] * fb);
+            w[4 * j + 3] = __float_as_uint(o[4 * j + 3] * fb);
           }
-          tmem_st16(tmem_base + lane_addr + c, o);
+          tmem_st16x256_x8(tmem_base + lane_addr + c, w);
         }
         tmem_wait_st();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_empty);
       // P = 2^(s - m) in bf16; the sums add the rounded values PV actually uses
       uint32_t pa[8], pb[8];
 #pragma unroll
@@ -376,11 +467,11 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         if (!(ok = mbar_wait_warp(o_done, (it - 1) & 1, abort_flag))) break;  // P buffer free
       }
       {
-        const int ha = sw * 16 + ra, hb = ha + 8;
+        const int ha = sw * 16 + ra, hbr = ha + 8;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(ha, j) + 2 * cc) = pa[j];
-          *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(hb, j) + 2 * cc) = pb[j];
+          *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(hbr, j) + 2 * cc) = pb[j];
         }
       }
       fence_proxy_async_smem();
@@ -393,33 +484,33 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
     // hand (max, sum) of head row r to O lane r (the 32-lane layout below)
-    float m_used, l;
+    float m_h, l_h;
     {
       const int src = 4 * (lane & 7);
       const float xa = __shfl_sync(0xffffffffu, m_a, src), xb = __shfl_sync(0xffffffffu, m_b, src);
       const float ya = __shfl_sync(0xffffffffu, l_a, src), yb = __shfl_sync(0xffffffffu, l_b, src);
-      m_used = ((lane & 15) < 8) ? xa : xb;
-      l = ((lane & 15) < 8) ? ya : yb;
+      m_h = ((lane & 15) < 8) ? xa : xb;
+      l_h = ((lane & 15) < 8) ? ya : yb;
     }
     if (ok) ok = mbar_wait_warp(o_done, (n_tiles - 1) & 1, abort_flag);
-    const float l_h = l;        // lane r < 16 owns O row r; lanes 16..31 mirror it
-    const float m_h = m_used;
+    const bool o_row = lane < 16;               // lane r < 16 owns O row r
+    const int h_local = sw * 16 + (lane & 15);
     const int h = h0 + h_local;
     if (ok) tc_fence_after();
     if (S == 1) {
       if (ok) {
-        const bool writer = !is_s && h < p.H;
+        const bool writer = o_row && h < p.H;
         const float inv = (l_h > 0.0f) ? 1.0f / l_h : 0.0f;
         const int64_t row = static_cast<int64_t>(t) * p.H + h;
         for (int c = 0; c < DC; c += 16) {
-          float v[16];
-          tmem_ld16(tmem_base + lane_addr + c, v);
+          float o[16];
+          tmem_ld16(tmem_base + lane_addr + c, o);
           tmem_wait_ld();
           if (writer) {
             uint32_t w8[8];
 #pragma unroll
             for (int u = 0; u < 16; u += 2) {
-              const __nv_bfloat162 o2 = __floats2bfloat162_rn(v[u] * inv, v[u + 1] * inv);
+              const __nv_bfloat162 o2 = __floats2bfloat162_rn(o[u] * inv, o[u + 1] * inv);
               w8[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
             }
             uint4* dst = reinterpret_cast<uint4*>(p.out + row * DC + c);
@@ -429,92 +520,102 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         }
         if (writer && p.lse) p.lse[row] = (l_h > 0.0f) ? (m_h + log2f(l_h)) * 0.69314718055994531f : -INFINITY;
       }
-    } else {
-      // ---------------- merge the S split partials inside the cluster
-      // Head row h_local belongs to CTA owner = h_local % S (slot h_local / S).
-      // Each CTA sends its unnormalised O row with (running max, running sum)
-      // into the owner's buffer (entry src * HPC + slot); the owner combines.
-      const uint32_t me = cluster_ctarank();
-      const int HPC = (64 + S - 1) / S;
-      const uint32_t recv_base = smem_u32(smem + C::OFF_KV);
-      const uint32_t stat_base = smem_u32(smem + C::OFF_P);
-      if (ok && threadIdx.x == 0) {
-        // this CTA's loop is done (all PV products complete, no TMA in flight):
-        // its KV ring and P tile may now be overwritten by peers
-        for (int r = 0; r < S; ++r) mbar_arrive_remote(mapa_shared(smem_u32(ready), r));
-      }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(ready, 0, abort_flag));
-      if (ok) {
-        const uint32_t owner = static_cast<uint32_t>(h_local % S);
-        const int entry = static_cast<int>(me) * HPC + h_local / S;
-        const uint32_t o_dst = mapa_shared(recv_base + entry * DC * 4, owner);
-        for (int c = 0; c < DC; c += 16) {
-          float v[16];
-          tmem_ld16(tmem_base + lane_addr + c, v);
-          tmem_wait_ld();
-          if (!is_s) {
+    } else if (ok) {
+      // this split's unnormalised rows and statistics -> workspace (L2). A
+      // partial block is stored as [column / 4][head row][4 floats], so the
+      // 16 rows of a warp write 256 contiguous bytes per store.
+      const int64_t grp = (static_cast<int64_t>(t) * gridDim.y + hb) * S;
+      float4* po = reinterpret_cast<float4*>(p.part_o + (grp + split) * C::HB * DC) + h_local;
+#pragma unroll 1
+      for (int c = 0; c < DC; c += 32) {
+        float o[16], o2[16];
+        tmem_ld16(tmem_base + lane_addr + c, o);
+        tmem_ld16(tmem_base + lane_addr + c + 16, o2);
+        tmem_wait_ld();
+        if (o_row) {
 #pragma unroll
-            for (int u = 0; u < 16; u += 4) st_cluster_v4(o_dst + (c + u) * 4, v[u], v[u + 1], v[u + 2], v[u + 3]);
-          }
-        }
-        if (!is_s) {
-          st_cluster_v2(mapa_shared(stat_base + entry * 8, owner), m_h, l_h);
-          // 64 O-row threads per CTA arrive on every CTA's recv barrier (count
-          // 64 * S); release order makes each thread's stores visible first
-          for (int r = 0; r < S; ++r) mbar_arrive_remote(mapa_shared(smem_u32(recv), r));
-        }
-      }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait_cluster(recv, 0, abort_flag));
-      if (ok) {
-        // finalise the heads this CTA owns: warp sw takes slots sw, sw+4, ...
-        const float* obuf = reinterpret_cast<const float*>(smem + C::OFF_KV);
-        const float2* sbuf = reinterpret_cast<const float2*>(smem + C::OFF_P);
-        for (int slot = sw; slot < HPC; slot += 4) {
-          const int hl = slot * S + static_cast<int>(me);
-          if (hl >= 64 || h0 + hl >= p.H) continue;
-          float M = -INFINITY;
-          for (int src = 0; src < S; ++src) M = fmaxf(M, sbuf[src * HPC + slot].x);
-          float L = 0.0f;
-          for (int src = 0; src < S; ++src) {
-            const float2 st = sbuf[src * HPC + slot];
-            if (st.y > 0.0f) L += exp2f(st.x - M) * st.y;
-          }
-          const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-          const int64_t row = static_cast<int64_t>(t) * p.H + h0 + hl;
-          for (int d0 = lane * 8; d0 < DC; d0 += 32 * 8) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int src = 0; src < S; ++src) {
-              const float2 st = sbuf[src * HPC + slot];
-              if (!(st.y > 0.0f)) continue;
-              const float wgt = exp2f(st.x - M) * inv;
-              const float4* o4 = reinterpret_cast<const float4*>(obuf + (src * HPC + slot) * DC + d0);
-              const float4 a = o4[0], c4 = o4[1];
-              acc[0] = fmaf(wgt, a.x, acc[0]);
-              acc[1] = fmaf(wgt, a.y, acc[1]);
-              acc[2] = fmaf(wgt, a.z, acc[2]);
-              acc[3] = fmaf(wgt, a.w, acc[3]);
-              acc[4] = fmaf(wgt, c4.x, acc[4]);
-              acc[5] = fmaf(wgt, c4.y, acc[5]);
-              acc[6] = fmaf(wgt, c4.z, acc[6]);
-              acc[7] = fmaf(wgt, c4.w, acc[7]);
-            }
-            uint32_t w4[4];
+          for (int u = 0; u < 4; ++u)
+            po[(c / 4 + u) * C::HB] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
 #pragma unroll
-            for (int u = 0; u < 8; u += 2) {
-              const __nv_bfloat162 o2 = __floats2bfloat162_rn(acc[u], acc[u + 1]);
-              w4[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
-            }
-            *reinterpret_cast<uint4*>(p.out + row * DC + d0) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-          if (lane == 0 && p.lse) p.lse[row] = (L > 0.0f) ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+          for (int u = 0; u < 4; ++u)
+            po[(c / 4 + 4 + u) * C::HB] = make_float4(o2[4 * u], o2[4 * u + 1], o2[4 * u + 2], o2[4 * u + 3]);
         }
       }
+      if (o_row) p.part_ml[(grp + split) * C::HB + h_local] = make_float2(m_h, l_h);
+    }
+  }
+
+  if (S > 1) {
+    // ---------------- merge the key-split partials through global memory
+    // The cluster barrier (release/acquire at cluster scope) orders every
+    // CTA's partial writes before any CTA reads them. Head h_local is
+    // finalised by split h_local % S, the work spread over all threads.
+    cluster_sync_all();
+    const int64_t grp = (static_cast<int64_t>(t) * gridDim.y + hb) * S;
+    constexpr int SL = 16;                     // columns per item
+    constexpr int NSL = DC / SL;
+    const int owned = (C::HB - split + S - 1) / S;  // heads split, split + S, ...
+    // consecutive threads take consecutive owned heads of one slice, so the
+    // [column / 4][head row] partial layout is read in 16-byte runs; splits
+    // are folded in with a running maximum, so every load of an item is
+    // issued before any of its arithmetic
+    for (int item = threadIdx.x; item < owned * NSL; item += C::THREADS) {
+      const int hl = split + S * (item % owned);
+      const int c0 = (item / owned) * SL;
+      const int h = h0 + hl;
+      if (h >= p.H) continue;
+      float Mx = -INFINITY, L = 0.0f;
+      float acc[SL];
+#pragma unroll
+      for (int u = 0; u < SL; ++u) acc[u] = 0.0f;
+      for (int sb = 0; sb < S; sb += 2) {
+        float2 ml[2];
+        float4 x[2][SL / 4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (sb + u < S) {
+            ml[u] = __ldcg(&p.part_ml[(grp + sb + u) * C::HB + hl]);
+            const float4* po = reinterpret_cast<const float4*>(p.part_o + (grp + sb + u) * C::HB * DC) + hl;
+#pragma unroll
+            for (int v4 = 0; v4 < SL / 4; ++v4) x[u][v4] = __ldcg(po + (c0 / 4 + v4) * C::HB);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (sb + u < S && ml[u].y > 0.0f) {
+            const float nm = fmaxf(Mx, ml[u].x);
+            const float fo = exp2f(Mx - nm);       // 0 while nothing is accumulated (Mx = -inf)
+            const float fn = exp2f(ml[u].x - nm);
+            L = L * fo + ml[u].y * fn;
+#pragma unroll
+            for (int v4 = 0; v4 < SL / 4; ++v4) {
+              acc[4 * v4 + 0] = acc[4 * v4 + 0] * fo + x[u][v4].x * fn;
+              acc[4 * v4 + 1] = acc[4 * v4 + 1] * fo + x[u][v4].y * fn;
+              acc[4 * v4 + 2] = acc[4 * v4 + 2] * fo + x[u][v4].z * fn;
+              acc[4 * v4 + 3] = acc[4 * v4 + 3] * fo + x[u][v4].w * fn;
+            }
+            Mx = nm;
+          }
+        }
+      }
+      const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+      const int64_t row = static_cast<int64_t>(t) * p.H + h;
+      uint32_t w[SL / 2];
+#pragma unroll
+      for (int u = 0; u < SL; u += 2) {
+        const __nv_bfloat162 o2 = __floats2bfloat162_rn(acc[u] * inv, acc[u + 1] * inv);
+        w[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * DC + c0);
+#pragma unroll
+      for (int u = 0; u < SL / 8; ++u) dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      if (c0 == 0 && p.lse) p.lse[row] = (L > 0.0f) ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }

@@ -112,8 +112,8 @@ def test_mla_validation(lib):
     assert call(_mla_in(), out=MIS) == B.DSA_ERR_MISALIGNED
     assert call(_mla_in(), k=0) == B.DSA_ERR_UNSUPPORTED_SHAPE
     assert call(_mla_in(), k=4096) == B.DSA_ERR_UNSUPPORTED_SHAPE
-    # split partials merge inside a cluster: the attention takes no workspace
-    assert lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128) == 0
+    # key-split partials merge through the workspace; a tiny batch splits its keys
+    assert lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128) > 0
 
 
 def test_fused_and_quant_validation(lib):
