@@ -207,6 +207,7 @@ def main():
     from indexed_sparse_attention_relu_b200 import binding as B
     from indexed_sparse_attention_relu_b200 import build as build_mod
     from indexed_sparse_attention_relu_b200 import device as DV
+    from indexed_sparse_attention_relu_b200 import multi
     from indexed_sparse_attention_relu_b200 import workloads as W
 
     if not torch.cuda.is_available():
@@ -299,12 +300,10 @@ def main():
         "topk": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
         "sparse_mla": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
     }
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    # the job's time is its slowest rank's; every rank ran its own T queries
+    total_ms = multi.max_over_ranks(total_ms, dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step * 1e-3)
+    value = multi.job_throughput([T] * world, ms_per_step)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies timed
     h_qidx = base.q_idx.cpu().pin_memory()
@@ -334,10 +333,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = multi.max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
     status2 = B.dsa_read_device_status(stream)
 
     # ---- roofline of the dominant stage
