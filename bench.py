@@ -18,6 +18,7 @@ records on its stream between its stages.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -343,12 +344,20 @@ def main():
     peak, peak_kind = _peaks()
     achieved = algo[dom] / (stage_ms[dom] * 1e-3) / 1e9
     step_gbs = algo["step"] / (ms_per_step * 1e-3) / 1e9
+    # DRAM bytes per launch of the dominant kernel from the committed ncu
+    # capture, used only while the kernel's sources are the ones it measured
     traffic = None
-    prof = os.path.join(ROOT, "profiles", f"dram_traffic_{args.config}.json")
+    prof = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if os.path.exists(prof):
         try:
-            traffic = json.load(open(prof)).get(dom)
-        except Exception:
+            rec = json.load(open(prof)).get(dom)
+            if rec and rec.get("workload") == args.config:
+                h = hashlib.sha256()
+                for src in rec["sources"]:
+                    h.update(open(os.path.join(ROOT, src), "rb").read())
+                if h.hexdigest() == rec["sources_sha256"]:
+                    traffic = rec["dram_bytes_read"] + rec["dram_bytes_write"]
+        except (OSError, KeyError, ValueError):
             traffic = None
 
     # kernels launched per step: indexer, Top-K, attention (split partials merge
