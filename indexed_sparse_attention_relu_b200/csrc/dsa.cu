@@ -298,19 +298,25 @@ dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int
   p.L_max = bt->max_seq_len;
   p.K = k;
   p.idx = idx;
+  p.bm_words = 0;
   const int L = bt->max_seq_len;
-  // rows of up to 1024 * IPT candidates: register/shared-memory resident select
-  if (L <= 1024 * 8) {
-    p.cache_cap = 1024 * 8;
-    return launch_topk_kernel(topk_row_kernel<1024, 8>, 1024, 1024 * 8 * 4, p, bt->num_q, st, pdl);
-  }
-  if (L <= 1024 * 16) {
-    p.cache_cap = 1024 * 16;
-    return launch_topk_kernel(topk_row_kernel<1024, 16>, 1024, 1024 * 16 * 4, p, bt->num_q, st, pdl);
-  }
-  if (L <= 1024 * 32) {
-    p.cache_cap = 1024 * 32;
-    return launch_topk_kernel(topk_row_kernel<1024, 32>, 1024, 1024 * 32 * 4, p, bt->num_q, st, pdl);
+  // two streaming passes with position bitmaps in shared memory: the bitmaps
+  // and first-digit histogram are fixed; the candidate list of the threshold
+  // bin gets a quarter of a row (at least 2048, at most 16384 slots) within
+  // the shared-memory budget (a longer list streams the row instead)
+  {
+    const int bm_words = ((L + 31) / 32 + 1) & ~1;
+    const int fixed = 4 * 2048 * 4 + 2 * bm_words * 4;
+    const int budget = 232448 - 6144 - fixed;  // static shared memory of the kernel included
+    int cap = L / 4;
+    if (cap < 2048) cap = 2048;
+    if (cap > 16384) cap = 16384;
+    if (cap * 8 > budget) cap = budget / 8;
+    if (cap >= 1024) {
+      p.bm_words = bm_words;
+      p.cache_cap = cap;
+      return launch_topk_kernel(topk_bitmap_kernel<1024>, 1024, fixed + cap * 8, p, bt->num_q, st, pdl);
+    }
   }
   // longer rows: multi-pass select streaming the row from L2 / HBM
   const int cap = L < kTopkCacheMax ? L : kTopkCacheMax;

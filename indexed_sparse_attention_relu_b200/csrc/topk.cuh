@@ -6,15 +6,14 @@
 // its n_valid(t) = min(q_pos + 1, seq_len) causal candidates; fewer than K
 // candidates -> all of them, padded with -1. Output ascending by position.
 //
-// Method: scores map to order-preserving uint32 keys (-0 == +0). One CTA per
-// row finds the K-th largest key tau with four 8-bit most-significant-digit
-// histogram passes (warp-aggregated shared atomics), which also yields
-// `need` = how many keys equal to tau must be taken. A final pass walks the
-// row in position order with two block-wide exclusive scans: the first ranks
-// the keys equal to tau (the lowest positions win), the second places every
-// selected position, so the output comes out sorted with no sort. Rows that
-// fit in shared memory are cached there; longer rows are re-read from L2/HBM
-// on each pass. The result depends only on the scores (bit-deterministic).
+// Method: scores map to order-preserving uint32 keys (-0 == +0); one CTA per
+// row finds the K-th largest key tau and `need` = how many keys equal to tau
+// must be taken (the lowest positions win). topk_bitmap_kernel (every row
+// whose position bitmaps fit in shared memory) needs two streaming passes
+// over the row; topk_kernel (longer rows) one pass per 8-bit radix digit.
+// Both emit the selected positions in position order with two block-wide
+// exclusive scans, so the output comes out sorted with no sort. The result
+// depends only on the scores (bit-deterministic).
 #pragma once
 #include <cub/block/block_scan.cuh>
 
@@ -32,7 +31,9 @@ struct TopkParams {
   int32_t L_max;
   int32_t K;
   int32_t* idx;
-  int32_t cache_cap;  // keys that fit in the dynamic shared-memory cache
+  int32_t cache_cap;  // keys that fit in the dynamic shared-memory cache (radix kernels),
+                      // candidate slots of the threshold bin (bitmap kernel)
+  int32_t bm_words;   // words of each position bitmap (bitmap kernel): >= ceil(L_max / 32), even
 };
 
 template <int THREADS>
@@ -189,22 +190,71 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Rows of up to THREADS * IPT candidates (decode and most prefill rows).
-// Thread i owns the contiguous positions [i*IPT, (i+1)*IPT): its keys are
-// cached in shared memory, every radix pass adds into a per-warp histogram
-// (conflicts only inside a warp), 256 threads reduce and scan the 256 bins in
-// parallel, and the final emission needs just two block-wide scans because
-// ownership is already in position order.
-template <int THREADS, int IPT>
-__global__ void __launch_bounds__(THREADS, 1) topk_row_kernel(const TopkParams p) {
-  static_assert(IPT % 4 == 0, "IPT must be a multiple of 4");
-  constexpr int WARPS = THREADS / 32;
+// Rows of any length whose position bitmaps fit in shared memory: two
+// streaming passes over the row instead of one pass per radix digit.
+//  A. Histogram of the top 11 key bits (2048 bins, four copies against
+//     atomic contention); a block scan from the top bin down finds the bin
+//     b* that holds the K-th largest key and the count `above` of keys in
+//     higher bins.
+//  B. Every position in a higher bin is selected: its bit is set in the
+//     selection bitmap (a warp covers 32 aligned positions, so it writes whole
+//     words). Keys in b* are appended (key, position) to a candidate list.
+// The K - above largest candidates are found with radix passes over the 21
+// remaining key bits (on the candidate list; by streaming the row restricted
+// to b* when the list overflowed), giving the K-th largest key tau and the
+// number `need` of keys equal to tau to take (the lowest positions). Keys
+// above tau join the selection bitmap, keys equal to tau an "equal" bitmap.
+// Emission walks the bitmaps in position order with two block scans (the
+// first ranks the equal keys, the second places the outputs), so the indices
+// come out ascending with no sort.
+template <int THREADS>
+__device__ __forceinline__ void topk_find_digit(const uint32_t* h256, int width, int& kr, int* wsum, int* s_digit,
+                                                int* s_krem) {
+  // bins in descending digit order among the 2^width used ones; threads 0..255
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  int cnt = 0, incl = 0;
+  if (tid < 256) {
+    const int d = 255 - tid;
+    cnt = (d < (1 << width)) ? static_cast<int>(h256[d]) : 0;
+    incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+  }
+  __syncthreads();
+  if (tid < 256) {
+    int before = 0;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    incl += before;
+    const int excl = incl - cnt;
+    if (excl < kr && kr <= incl) {
+      *s_digit = 255 - tid;
+      *s_krem = kr - excl;
+    }
+  }
+  __syncthreads();
+  kr = *s_krem;
+}
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, 1) topk_bitmap_kernel(const TopkParams p) {
+  constexpr int HBITS = 11;
+  constexpr int NB = 1 << HBITS;
+  constexpr int HCOPIES = 4;
+  constexpr int LOW = 32 - HBITS;  // key bits below the first digit
+  static_assert(2 * THREADS == NB, "two first-digit bins per thread");
   using Scan = cub::BlockScan<int, THREADS>;
   __shared__ typename Scan::TempStorage scan_tmp;
-  __shared__ int whist[WARPS][256];
   __shared__ int wsum[8];
-  __shared__ int sel_digit, sel_krem;
-  extern __shared__ __align__(16) uint32_t keys[];  // THREADS * IPT
+  __shared__ int s_bin, s_above, s_ncand, s_digit, s_krem;
+  extern __shared__ __align__(16) uint32_t sm[];
+  uint32_t* hist = sm;                                         // [HCOPIES][NB]
+  uint32_t* selb = hist + HCOPIES * NB;                        // [bm_words]
+  uint32_t* eqb = selb + p.bm_words;                           // [bm_words]
+  uint2* cands = reinterpret_cast<uint2*>(eqb + p.bm_words);   // [cache_cap] (key, position)
 
   const int t = blockIdx.x;
   const int tid = threadIdx.x;
@@ -215,135 +265,157 @@ __global__ void __launch_bounds__(THREADS, 1) topk_row_kernel(const TopkParams p
   const int n = max(0, min(__ldg(p.q_pos + t) + 1, len));
   int32_t* out = p.idx + static_cast<int64_t>(t) * p.K;
   const float* row = p.scores + static_cast<int64_t>(t) * p.ld;
-  pdl_launch_dependents();
-  pdl_wait_prior();
+  pdl_launch_dependents();  // the attention may be scheduled; it waits for these indices
+  pdl_wait_prior();         // the indexer's scores (and anything before it) are complete
 
   if (n <= p.K) {
     for (int i = tid; i < p.K; i += THREADS) out[i] = (i < n) ? i : -1;
     return;
   }
-  for (int i = tid; i < WARPS * 256; i += THREADS) (&whist[0][0])[i] = 0;
+  const int nw = (n + 31) >> 5;
+  for (int i = tid; i < HCOPIES * NB; i += THREADS) hist[i] = 0u;
+  for (int i = tid; i < nw; i += THREADS) {
+    selb[i] = 0u;
+    eqb[i] = 0u;
+  }
+  if (tid == 0) s_ncand = 0;
+  __syncthreads();
 
-  // ---- load this thread's contiguous positions (all loads in flight at once)
-  const int base = tid * IPT;
+  // ---- A: first-digit histogram (four independent loads in flight per thread)
   {
-    float v[IPT];
-    const bool vec = ((p.ld & 3) == 0) && ((reinterpret_cast<uintptr_t>(p.scores) & 15) == 0);
-    if (vec && base + IPT <= n) {
+    uint32_t* myh = hist + (warp & (HCOPIES - 1)) * NB;
+    for (int i0 = tid; i0 < n; i0 += 4 * THREADS) {
+      float v[4];
 #pragma unroll
-      for (int u = 0; u < IPT; u += 4) {
-        const float4 f = ld_dep4(row + base + u);
-        v[u] = f.x;
-        v[u + 1] = f.y;
-        v[u + 2] = f.z;
-        v[u + 3] = f.w;
+      for (int u = 0; u < 4; ++u) v[u] = (i0 + u * THREADS < n) ? ld_dep(row + i0 + u * THREADS) : 0.0f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + u * THREADS < n) atomicAdd(&myh[float_order_key(v[u]) >> LOW], 1u);
+    }
+  }
+  __syncthreads();
+  {
+    const int b1 = NB - 1 - 2 * tid, b2 = b1 - 1;
+    int h1 = 0, h2 = 0;
+#pragma unroll
+    for (int c = 0; c < HCOPIES; ++c) {
+      h1 += static_cast<int>(hist[c * NB + b1]);
+      h2 += static_cast<int>(hist[c * NB + b2]);
+    }
+    int before;
+    Scan(scan_tmp).ExclusiveSum(h1 + h2, before);
+    if (before < p.K && p.K <= before + h1 + h2) {
+      if (before + h1 >= p.K) {
+        s_bin = b1;
+        s_above = before;
+      } else {
+        s_bin = b2;
+        s_above = before + h1;
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t bstar = static_cast<uint32_t>(s_bin);
+  int kr = p.K - s_above;  // keys to take from bin b*
+
+  // ---- B: positions in higher bins -> selection bitmap; keys in b* -> candidates
+  for (int i0 = warp * 32; i0 < n; i0 += THREADS) {
+    const int i = i0 + lane;
+    const bool valid = i < n;
+    const uint32_t key = valid ? float_order_key(ld_dep(row + i)) : 0u;
+    const uint32_t kb = key >> LOW;
+    const unsigned selmask = __ballot_sync(0xffffffffu, valid && kb > bstar);
+    if (lane == 0 && selmask) selb[i0 >> 5] = selmask;
+    const unsigned cmask = __ballot_sync(0xffffffffu, valid && kb == bstar);
+    if (cmask) {
+      int base = 0;
+      if (lane == 0) base = atomicAdd(&s_ncand, __popc(cmask));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if ((cmask >> lane) & 1u) {
+        const int slot = base + __popc(cmask & ((1u << lane) - 1u));
+        if (slot < p.cache_cap) cands[slot] = make_uint2(key, static_cast<uint32_t>(i));
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- exact threshold inside b*: digits of 8, 8 and 5 bits
+  const int ncand = s_ncand;
+  const bool listed = ncand <= p.cache_cap;
+  uint32_t prefix = bstar << LOW, mask = ~0u << LOW;
+  uint32_t* h256 = hist;  // reuse
+  const int shifts[3] = {LOW - 8, LOW - 16, 0};
+  const int widths[3] = {8, 8, LOW - 16};
+#pragma unroll 1
+  for (int ps = 0; ps < 3; ++ps) {
+    const int shift = shifts[ps];
+    const uint32_t wm = (1u << widths[ps]) - 1u;
+    if (tid < 256) h256[tid] = 0u;
+    __syncthreads();
+    if (listed) {
+      for (int c = tid; c < ncand; c += THREADS) {
+        const uint32_t key = cands[c].x;
+        if ((key & mask) == prefix) atomicAdd(&h256[(key >> shift) & wm], 1u);
       }
     } else {
-#pragma unroll
-      for (int u = 0; u < IPT; ++u) v[u] = (base + u < n) ? ld_dep(row + base + u) : 0.0f;
+      for (int i = tid; i < n; i += THREADS) {
+        const uint32_t key = float_order_key(ld_dep(row + i));
+        if ((key & mask) == prefix) atomicAdd(&h256[(key >> shift) & wm], 1u);
+      }
     }
-#pragma unroll
-    for (int u = 0; u < IPT; u += 4) {
-      uint4 k4;
-      k4.x = (base + u + 0 < n) ? float_order_key(v[u + 0]) : 0u;
-      k4.y = (base + u + 1 < n) ? float_order_key(v[u + 1]) : 0u;
-      k4.z = (base + u + 2 < n) ? float_order_key(v[u + 2]) : 0u;
-      k4.w = (base + u + 3 < n) ? float_order_key(v[u + 3]) : 0u;
-      *reinterpret_cast<uint4*>(keys + base + u) = k4;
+    __syncthreads();
+    topk_find_digit<THREADS>(h256, widths[ps], kr, wsum, &s_digit, &s_krem);
+    prefix |= static_cast<uint32_t>(s_digit) << shift;
+    mask |= wm << shift;
+  }
+  const uint32_t tau = prefix;  // the K-th largest key
+  const int need = kr;          // keys equal to tau that are taken (lowest positions first)
+  if (listed) {
+    for (int c = tid; c < ncand; c += THREADS) {
+      const uint2 kp = cands[c];
+      if (kp.x > tau) atomicOr(&selb[kp.y >> 5], 1u << (kp.y & 31));
+      else if (kp.x == tau) atomicOr(&eqb[kp.y >> 5], 1u << (kp.y & 31));
+    }
+  } else {
+    for (int i = tid; i < n; i += THREADS) {
+      const uint32_t key = float_order_key(ld_dep(row + i));
+      if ((key >> LOW) != bstar) continue;
+      if (key > tau) atomicOr(&selb[i >> 5], 1u << (i & 31));
+      else if (key == tau) atomicOr(&eqb[i >> 5], 1u << (i & 31));
     }
   }
-  const int mine = max(0, min(IPT, n - base));  // valid positions owned by this thread
   __syncthreads();
 
-  uint32_t prefix = 0u, mask = 0u;
-  int krem = p.K;
-#pragma unroll 1
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-#pragma unroll
-    for (int u = 0; u < IPT; u += 4) {
-      const uint4 k4 = *reinterpret_cast<const uint4*>(keys + base + u);
-      const uint32_t kk[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (u + j < mine && (kk[j] & mask) == prefix) atomicAdd(&whist[warp][(kk[j] >> shift) & 0xFFu], 1);
-    }
-    __syncthreads();
-    // 256 threads: bin total (descending digit order), reset, inclusive scan
-    int cnt = 0, incl = 0;
-    if (tid < 256) {
-      const int d = 255 - tid;
-#pragma unroll 4
-      for (int w = 0; w < WARPS; ++w) {
-        cnt += whist[w][d];
-        whist[w][d] = 0;
-      }
-      incl = cnt;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      if (lane == 31) wsum[warp] = incl;
-    }
-    __syncthreads();
-    if (tid < 256) {
-      int before_warp = 0;
-      for (int w = 0; w < warp; ++w) before_warp += wsum[w];
-      incl += before_warp;
-      const int excl = incl - cnt;
-      if (excl < krem && krem <= incl) {
-        sel_digit = 255 - tid;
-        sel_krem = krem - excl;
-      }
-    }
-    __syncthreads();
-    prefix |= static_cast<uint32_t>(sel_digit) << shift;
-    mask |= 0xFFu << shift;
-    krem = sel_krem;
+  // ---- emission in position order
+  const int wpt = (nw + THREADS - 1) / THREADS;
+  const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
+  int cs = 0, ce = 0;
+  for (int w = w0; w < w1; ++w) {
+    cs += __popc(selb[w]);
+    ce += __popc(eqb[w]);
   }
-  const uint32_t tau = prefix;   // the K-th largest key
-  const int need = krem;         // keys equal to tau that are taken (lowest positions first)
-
-  int n_eq = 0;
-#pragma unroll
-  for (int u = 0; u < IPT; ++u) n_eq += (u < mine && keys[base + u] == tau) ? 1 : 0;
-  int eq_before, eq_total;
-  Scan(scan_tmp).ExclusiveSum(n_eq, eq_before, eq_total);
+  int eq_before;
+  Scan(scan_tmp).ExclusiveSum(ce, eq_before);
   __syncthreads();
-  int n_sel = 0;
-  {
-    int e = eq_before;
-#pragma unroll
-    for (int u = 0; u < IPT; ++u) {
-      if (u >= mine) break;
-      const uint32_t k = keys[base + u];
-      if (k > tau) {
-        ++n_sel;
-      } else if (k == tau) {
-        n_sel += (e < need) ? 1 : 0;
+  const int take_eq = max(0, min(ce, need - eq_before));
+  int out_before;
+  Scan(scan_tmp).ExclusiveSum(cs + take_eq, out_before);
+  int o = out_before, e = eq_before;
+  for (int w = w0; w < w1; ++w) {
+    const uint32_t sb = selb[w], eb = eqb[w];
+    uint32_t all = sb | eb;
+    while (all) {
+      const int bit = __ffs(all) - 1;
+      all &= all - 1u;
+      const int pos = w * 32 + bit;
+      if ((sb >> bit) & 1u) {
+        if (o < p.K) out[o++] = pos;
+      } else {
+        if (e < need && o < p.K) out[o++] = pos;
         ++e;
       }
     }
   }
-  int out_before, out_total;
-  Scan(scan_tmp).ExclusiveSum(n_sel, out_before, out_total);
-  {
-    int e = eq_before, o = out_before;
-#pragma unroll
-    for (int u = 0; u < IPT; ++u) {
-      if (u >= mine) break;
-      const uint32_t k = keys[base + u];
-      bool take = k > tau;
-      if (k == tau) {
-        take = e < need;
-        ++e;
-      }
-      if (take && o < p.K) out[o++] = base + u;
-    }
-  }
-  (void)eq_total;
-  (void)out_total;
 }
 
 }  // namespace dsa

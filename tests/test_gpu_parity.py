@@ -169,14 +169,22 @@ def test_topk_tie_cases():
     assert list(idx[2][:40]) == list(range(40)) and np.all(idx[2][40:] == -1)
 
 
-def test_topk_long_rows_uncached():
-    """Rows longer than the shared-memory cache take the streaming path."""
+def test_topk_long_rows_and_crowded_threshold_bin():
+    """Long rows (two streaming passes), and rows whose threshold bin holds more
+    keys than the candidate list (all equal, or a constant bulk under a few
+    larger values): the exact threshold is then found by streaming the row
+    restricted to that bin."""
     rng = np.random.default_rng(7)
+    bulk = np.full(60_000, 0.75, np.float32)
+    bulk[rng.choice(60_000, 1000, replace=False)] = 2.0
     rows = [W.bf16_round(rng.standard_normal(70_000).astype(np.float32) * 8),
-            np.float32(rng.integers(-50, 50, 60_000))]
+            np.float32(rng.integers(-50, 50, 60_000)),
+            np.zeros(60_000, np.float32),
+            bulk]
     idx, sc, lens = _topk_rows(rows, 2048)
     want = oracle.topk(sc.astype(np.float64), lens, 2048)
     assert np.array_equal(idx, want)
+    assert list(idx[2]) == list(range(2048))
 
 
 # ----------------------------------------------------------------------------- sparse MLA
