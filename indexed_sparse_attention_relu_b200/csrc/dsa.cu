@@ -206,7 +206,7 @@ dsa_status set_smem(Kern k, int bytes) {
 
 template <int HI, int DIN, int G, bool FP8>
 dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool pdl) {
   using C = IndexerCfg<HI, DIN, G, FP8>;
   CUtensorMap map;
   dsa_status s = make_key_map(&map, in->k_cache, static_cast<int64_t>(bt->batch) * bt->max_seq_len, DIN, FP8);
@@ -240,27 +240,41 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   p.scores = scores;
   p.ld = ld;
   p.tiles_per_cta = tpc;
-  kern<<<dim3(groups, gy), C::THREADS, C::SMEM_BYTES, st>>>(map, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(groups, gy);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, map, p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "indexer launch: %s", cudaGetErrorString(e));
   return check_launch("indexer_scores");
 }
 
 template <int HI, int DIN>
 dsa_status launch_indexer_g(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool pdl) {
   const bool fp8 = in->key_dtype == DSA_KEY_FP8_E4M3;
   if (indexer_group(bt) == 4)
-    return fp8 ? launch_indexer_t<HI, DIN, 4, true>(bt, in, scores, ld, st)
-               : launch_indexer_t<HI, DIN, 4, false>(bt, in, scores, ld, st);
-  return fp8 ? launch_indexer_t<HI, DIN, 1, true>(bt, in, scores, ld, st)
-             : launch_indexer_t<HI, DIN, 1, false>(bt, in, scores, ld, st);
+    return fp8 ? launch_indexer_t<HI, DIN, 4, true>(bt, in, scores, ld, st, pdl)
+               : launch_indexer_t<HI, DIN, 4, false>(bt, in, scores, ld, st, pdl);
+  return fp8 ? launch_indexer_t<HI, DIN, 1, true>(bt, in, scores, ld, st, pdl)
+             : launch_indexer_t<HI, DIN, 1, false>(bt, in, scores, ld, st, pdl);
 }
 
+// pdl: launch with programmatic stream serialization, so the prologue may
+// overlap the tail of the previous kernel in the stream (the kernel itself
+// still completes only after that kernel, see its teardown).
 dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
-                          cudaStream_t st) {
-  if (in->n_heads == 64 && in->head_dim == 128) return launch_indexer_g<64, 128>(bt, in, scores, ld, st);
-  if (in->n_heads == 64 && in->head_dim == 32) return launch_indexer_g<64, 32>(bt, in, scores, ld, st);
-  if (in->n_heads == 4 && in->head_dim == 128) return launch_indexer_g<4, 128>(bt, in, scores, ld, st);
-  return launch_indexer_g<4, 32>(bt, in, scores, ld, st);
+                          cudaStream_t st, bool pdl = false) {
+  if (in->n_heads == 64 && in->head_dim == 128) return launch_indexer_g<64, 128>(bt, in, scores, ld, st, pdl);
+  if (in->n_heads == 64 && in->head_dim == 32) return launch_indexer_g<64, 32>(bt, in, scores, ld, st, pdl);
+  if (in->n_heads == 4 && in->head_dim == 128) return launch_indexer_g<4, 128>(bt, in, scores, ld, st, pdl);
+  return launch_indexer_g<4, 32>(bt, in, scores, ld, st, pdl);
 }
 
 constexpr int kTopkThreads = 512;
@@ -503,13 +517,14 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
     const cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), st);
     return e == cudaSuccess ? DSA_OK : fail(DSA_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
   };
-  if ((s = rec(0)) != DSA_OK) return s;
-  if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st)) != DSA_OK) return s;
-  if ((s = rec(1)) != DSA_OK) return s;
-  // Programmatic dependent launch on the two internal edges: each kernel's
-  // prologue overlaps the tail of the previous one and waits on the device
-  // for its results. Not used when stage events sit between the kernels.
+  // Programmatic dependent launch on every edge: each kernel's prologue
+  // overlaps the tail of the previous one (for the indexer: the previous
+  // call's attention) and waits on the device for what it consumes. Not used
+  // when stage events sit between the kernels.
   const bool pdl = stage_events == nullptr;
+  if ((s = rec(0)) != DSA_OK) return s;
+  if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st, pdl)) != DSA_OK) return s;
+  if ((s = rec(1)) != DSA_OK) return s;
   if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st, pdl)) != DSA_OK) return s;
   if ((s = rec(2)) != DSA_OK) return s;
   if ((s = launch_mla(batch, mla_in, idx, k, out, lse, static_cast<uint8_t*>(ws) + sc_bytes + id_bytes, mla_bytes, st,

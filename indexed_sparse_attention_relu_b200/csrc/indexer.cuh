@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   const int warp = warp_id();
   const int lane = lane_id();
   pdl_launch_dependents();  // the Top-K may be scheduled; it waits for these scores
+  if (threadIdx.x == 0) prefetch_tensormap(&kmap);
 
   // Single-token groups: the query rows depend only on the block index, so
   // their loads go out before the group lookup and overlap it.
@@ -174,35 +175,55 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
       misc[3] = tb;
       misc[4] = te;
       misc[6] = 0;
+      for (int i = 0; i < C::ST; ++i) {
+        mbar_init(&full[i], 1);
+        mbar_init(&empty[i], FP8 ? 4 : 1);
+      }
+      for (int i = 0; i < C::NACC; ++i) {
+        mbar_init(&acc_full[i], 1);
+        mbar_init(&acc_empty[i], 4);
+      }
+      for (int i = 0; i < C::CS; ++i) {
+        mbar_init(&conv_full[i], 4);
+        mbar_init(&conv_empty[i], 1);
+      }
+      mbar_init(drain, 1);
+      fence_mbar_init();
     }
   }
   __syncthreads();
   const int b = misc[0];
   const int tile_begin = misc[3];
   const int tile_end = misc[4];
-  if (b < 0 || tile_begin >= tile_end) return;  // uniform across the CTA
+  if (b < 0 || tile_begin >= tile_end) {  // uniform across the CTA
+    pdl_wait_prior();
+    return;
+  }
   const int t0 = misc[1];
   const int nt = misc[2];
   const int n_tiles = tile_end - tile_begin;
+  const int64_t row0 = static_cast<int64_t>(b) * p.L_max;
 
-  // ---- setup: barriers, query tile, head weights, TMEM
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < C::ST; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], FP8 ? 4 : 1);
+  // The first ST key tiles go out now (every stage starts empty), so their
+  // latency overlaps the query staging and the TMEM allocation below.
+  auto issue_tile = [&](int it) {
+    const int st = it % C::ST;
+    const int32_t y = static_cast<int32_t>(row0 + static_cast<int64_t>(tile_begin + it) * 128);
+    const uint32_t dst = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES);
+    if constexpr (FP8) {
+      mbar_arrive_expect_tx(&full[st], C::U8_TILE);
+      tma_load_2d(dst, &kmap, 0, y, &full[st]);
+    } else {
+      mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+#pragma unroll
+      for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384, &kmap, a * 64, y, &full[st]);
     }
-    for (int i = 0; i < C::NACC; ++i) {
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_empty[i], 4);
-    }
-    for (int i = 0; i < C::CS; ++i) {
-      mbar_init(&conv_full[i], 4);
-      mbar_init(&conv_empty[i], 1);
-    }
-    mbar_init(drain, 1);
-    fence_mbar_init();
-    prefetch_tensormap(&kmap);
-  }
+  };
+  const int prologue_tiles = min(n_tiles, C::ST);
+  if (threadIdx.x == 0)
+    for (int it = 0; it < prologue_tiles; ++it) issue_tile(it);
+
+  // ---- setup: query tile, head weights, TMEM
   // B operand: row n = (token g, head j) = g*HI + j; zero rows beyond the group / padding.
   {
     constexpr int CHUNKS_PER_ROW = C::DK / 8;
@@ -246,25 +267,15 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = static_cast<uint32_t>(misc[5]);
-  const int64_t row0 = static_cast<int64_t>(b) * p.L_max;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < n_tiles; ++it) {
+      int issued = prologue_tiles;
+      for (int it = prologue_tiles; it < n_tiles; ++it) {
         const int st = it % C::ST;
         if (!mbar_wait(&empty[st], ((it / C::ST) & 1) ^ 1, abort_flag)) break;
-        const int32_t y = static_cast<int32_t>(row0 + static_cast<int64_t>(tile_begin + it) * 128);
-        const uint32_t dst = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES);
-        if constexpr (FP8) {
-          mbar_arrive_expect_tx(&full[st], C::U8_TILE);
-          tma_load_2d(dst, &kmap, 0, y, &full[st]);
-        } else {
-          mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
-#pragma unroll
-          for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384, &kmap, a * 64, y, &full[st]);
-        }
+        issue_tile(it);
         ++issued;
       }
       // drain: every issued TMA load must land before the CTA can retire
@@ -425,6 +436,12 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  // Under programmatic dependent launch this grid may start while the
+  // previous kernel of the stream (the attention of the previous call) still
+  // runs. It reads nothing that kernel writes, but it must not complete
+  // before it: the next kernel (Top-K) waits only for this grid and then
+  // rewrites the indices the attention reads.
+  pdl_wait_prior();
 }
 
 }  // namespace dsa

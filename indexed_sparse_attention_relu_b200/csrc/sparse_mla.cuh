@@ -545,6 +545,10 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     }
   }
 
+  // The next kernel of the stream (the next call's indexer) may be scheduled
+  // now; it completes only after this grid (see the indexer's teardown).
+  pdl_launch_dependents();
+
   if (S > 1) {
     // ---------------- merge the key-split partials through global memory
     // The cluster barrier (release/acquire at cluster scope) orders every
