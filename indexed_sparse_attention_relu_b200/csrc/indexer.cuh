@@ -18,8 +18,9 @@
 // scores coalesced. FP8 keys are TMA-loaded as bytes and widened to bf16 in
 // shared memory by four converter warps (exact: every E4M3 value is a bf16).
 //
-// Roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner),
-// warps 2..5 = epilogue, warps 6..9 = FP8 converters (FP8 only).
+// Roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner), then the
+// epilogue warps (four; eight for multi-token groups, two per TMEM
+// sub-partition splitting the tokens), then four FP8 converters (FP8 only).
 #pragma once
 #include "dsa_common.cuh"
 
@@ -54,7 +55,10 @@ struct IndexerCfg {
   static constexpr int NACC = 2;                           // TMEM accumulator buffers
   static constexpr int TMEM_COLS = (NACC * N <= 32) ? 32 : (NACC * N <= 64) ? 64 : (NACC * N <= 128) ? 128
                                    : (NACC * N <= 256) ? 256 : 512;
-  static constexpr int NUM_WARPS = FP8 ? 10 : 6;
+  // epilogue warps: two per TMEM sub-partition for multi-token groups (each
+  // takes half of the tokens), one otherwise
+  static constexpr int EPI_WARPS = (G > 1 && HI % 64 == 0 && G % 2 == 0) ? 8 : 4;
+  static constexpr int NUM_WARPS = 2 + EPI_WARPS + (FP8 ? 4 : 0);
   static constexpr int THREADS = NUM_WARPS * 32;
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
@@ -181,7 +185,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
       }
       for (int i = 0; i < C::NACC; ++i) {
         mbar_init(&acc_full[i], 1);
-        mbar_init(&acc_empty[i], 4);
+        mbar_init(&acc_empty[i], C::EPI_WARPS);
       }
       for (int i = 0; i < C::CS; ++i) {
         mbar_init(&conv_full[i], 4);
@@ -320,9 +324,10 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
       volatile int never = 0;
       mbar_wait(drain, 0, &never);
     }
-  } else if (warp >= 2 && warp < 6) {
+  } else if (warp >= 2 && warp < 2 + C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int sub = warp & 3;                 // TMEM sub-partition this warp may access
+    const int part = (warp - 2) / 4;          // token half (eight epilogue warps) or 0
     const int r = sub * 32 + lane;            // key row inside the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     int nv[G];
@@ -350,6 +355,27 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
             if (g < G) score[g] = fmaf(w_s[col], fmaxf(v[c][u], 0.0f), score[g]);
           }
         }
+      } else if constexpr (HI % 64 == 0) {
+        // wide tiles, 64 heads per token: one token's 64 columns per TMEM
+        // round trip (four loads in flight, one wait); with eight epilogue
+        // warps each takes the columns of its half of the tokens
+        constexpr int COLS = C::EPI_WARPS == 8 ? C::N / 2 : C::N;
+#pragma unroll 1
+        for (int c = part * COLS; c < (part + 1) * COLS; c += 64) {
+          float v[4][16];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmem_ld16(tmem_base + lane_addr + acc * C::N + c + 16 * q, v[q]);
+          tmem_wait_ld();
+          float tok = 0.0f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 16; ++u) tok = fmaf(w_s[c + 16 * q + u], fmaxf(v[q][u], 0.0f), tok);
+          const int g = c / HI;
+#pragma unroll
+          for (int gg = 0; gg < G; ++gg)
+            if (gg == g) score[gg] += tok;
+        }
       } else {
         // wide tiles (HI >= 16): a 16-column chunk never straddles two tokens
         static_assert(HI % 16 == 0, "wide indexer tiles need HI % 16 == 0");
@@ -358,13 +384,13 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
           float v[16];
           tmem_ld16(tmem_base + lane_addr + acc * C::N + c, v);
           tmem_wait_ld();
-          float part = 0.0f;
+          float chunk = 0.0f;
 #pragma unroll
-          for (int u = 0; u < 16; ++u) part = fmaf(w_s[c + u], fmaxf(v[u], 0.0f), part);
+          for (int u = 0; u < 16; ++u) chunk = fmaf(w_s[c + u], fmaxf(v[u], 0.0f), chunk);
           const int g = c / HI;
 #pragma unroll
           for (int gg = 0; gg < G; ++gg)
-            if (gg == g) score[gg] += part;
+            if (gg == g) score[gg] += chunk;
         }
       }
       tc_fence_before();
@@ -376,9 +402,10 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
         if (s < p.L_max) sigma = __ldg(p.k_scale + row0 + s);
       }
       if (s < p.ld) {
+        constexpr int GPART = C::EPI_WARPS == 8 ? G / 2 : G;  // tokens this warp scores
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          if (g < nt) {
+          if (g < nt && g / GPART == part) {
             const float val = (s < nv[g]) ? score[g] * sigma : -INFINITY;
             p.scores[static_cast<int64_t>(t0 + g) * p.ld + s] = val;
           }
@@ -387,7 +414,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
     }
   } else if constexpr (FP8) {
     // ------------------------------------------------------------ FP8 -> bf16 converters
-    const int ct = threadIdx.x - 6 * 32;  // 0..127
+    const int ct = threadIdx.x - (2 + C::EPI_WARPS) * 32;  // 0..127
     constexpr int CPR = DIN / 16;         // 16-byte input chunks per key row
     for (int it = 0; it < n_tiles; ++it) {
       const int st = it % C::ST;
