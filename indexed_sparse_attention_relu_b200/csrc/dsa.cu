@@ -161,8 +161,8 @@ struct MlaPlan {
 // Key splits per (token, head block): enough CTAs to fill the SMs in one
 // wave, at most 8 (the splits of one (token, head block) form a cluster and
 // merge through distributed shared memory).
-MlaPlan mla_plan(int T, int HB, int K, int sms) {
-  const int tiles = (K + 63) / 64;
+MlaPlan mla_plan(int T, int HB, int K, int sms, int tk = 64) {
+  const int tiles = (K + tk - 1) / tk;
   const int base = T * HB;
   int splits = base >= sms ? 1 : sms / base;
   if (splits > 8) splits = 8;
@@ -170,7 +170,7 @@ MlaPlan mla_plan(int T, int HB, int K, int sms) {
   if (splits < 1) splits = 1;
   const int tps = (tiles + splits - 1) / splits;
   splits = (tiles + tps - 1) / tps;
-  return MlaPlan{splits, tps * 64};
+  return MlaPlan{splits, tps * tk};
 }
 
 // Workspace of the attention: with key splits, every split CTA leaves its
@@ -403,8 +403,12 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
 
 dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
                       void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false) {
-  const MlaPlan pl = mla_plan(bt->num_q, (in->n_heads + 63) / 64, k, num_sms());
-  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
+  const int hb = (in->n_heads + 63) / 64;
+  if (in->d_latent == 512) {
+    const MlaPlan pl = mla_plan(bt->num_q, hb, k, num_sms(), MlaCfg<576, 512>::TK);
+    return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
+  }
+  const MlaPlan pl = mla_plan(bt->num_q, hb, k, num_sms(), MlaCfg<80, 64>::TK);
   return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
 }
 

@@ -53,7 +53,7 @@ struct MlaParams {
   int32_t K;
   const int32_t* idx;        // [T, K]
   float scale_log2;          // softmax_scale * log2(e)
-  int32_t keys_per_split;    // multiple of 64
+  int32_t keys_per_split;    // multiple of the tile size
   int32_t splits;            // == cluster size along z
   __nv_bfloat16* out;        // [T, H, DC]
   float* lse;                // [T, H] or null
@@ -66,17 +66,24 @@ struct MlaCfg {
   static constexpr int DP = ((D + 63) / 64) * 64;   // K extent of the stored rows (whole atoms)
   static constexpr int AKQ = DP / 64;               // 128-byte atom columns per row
   static constexpr int HB = 64;                     // heads per CTA (MMA M)
-  static constexpr int TK = 64;                     // keys per tile (QK^T N, PV K)
+  // keys per tile (QK^T N, PV K) and gather stages. 80-key tiles (a QK^T
+  // instruction costs about the same at N = 80 as at N = 64) fit only two
+  // stages of 576-dim rows; measured slower (the gather then stalls the
+  // MMA), so three 64-key stages are used. The kernel supports both.
+  static constexpr int TK = 64;
+  static constexpr int NST = 3;
+  static constexpr int RPW = TK / 8;                // rows per gather warp
   static constexpr int KSTEPS = (D + 15) / 16;      // K steps of QK^T
-  static constexpr int ATOM_COL = 64 * 128;         // bytes of one atom column of a 64-row tile
+  static constexpr int ATOM_COL = TK * 128;         // bytes of one atom column of a TK-row tile
+  static constexpr int Q_ATOM = 64 * 128;           // bytes of one atom column of the 64-head Q tile
   static constexpr int KV_BYTES = TK * DP * 2;
   static constexpr int Q_BYTES = HB * DP * 2;       // staged in the last gather stage
-  static constexpr int P_BYTES = HB * TK * 2;
-  static constexpr int NST = 3;
+  static constexpr int P_ATOMS = (TK + 63) / 64;    // 64-key atom columns of P
+  static constexpr int P_BYTES = P_ATOMS * HB * 128;
   static constexpr int N_PV = DC < 256 ? DC : 256;
   static constexpr int PV_MMAS = DC / N_PV;
-  static constexpr uint32_t COL_S = 0;              // lane offset 16
-  static constexpr uint32_t COL_Q = 64;             // lane offset 16, DP/2 columns
+  static constexpr uint32_t COL_S = 0;              // lane offset 16, TK columns
+  static constexpr uint32_t COL_Q = ((TK + 63) / 64) * 64;  // lane offset 16, DP/2 columns
   static constexpr int TMEM_NEED = (DC > (int)COL_Q + DP / 2) ? DC : (int)COL_Q + DP / 2;
   static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
                                    : TMEM_NEED <= 256 ? 256 : 512;
@@ -93,6 +100,8 @@ struct MlaCfg {
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(64, TK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(64, N_PV, false, true);
   static_assert(DC % N_PV == 0 && DC % 64 == 0, "latent dim must be a multiple of 64");
+  static_assert(TK % 16 == 0 && (TK == 64 || TK == 80), "tile of 64 or 80 keys");
+  static_assert(ATOM_COL % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
   static_assert(TMEM_NEED <= 512, "TMEM budget");
   static_assert(Q_BYTES <= KV_BYTES, "Q is staged in one gather stage");
   static_assert((DP / 2) % 32 == 0, "Q columns come in 32-column groups");
@@ -121,6 +130,17 @@ __device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr, const uint32_t 
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
       "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
+}
+
+// 16 lanes x 256 bits, 2 repetitions (16 columns): the 16x256b register
+// layout of tmem_ld16x256_x8 for two 8-column repetitions.
+__device__ __forceinline__ void tmem_ld16x256_x2(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ uint2 ld_shared_v2u(uint32_t addr) {
@@ -214,22 +234,22 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     // the query block is an input of the call, not of the Top-K: load it now
     mbar_arrive_expect_tx(q_full, C::Q_BYTES);
 #pragma unroll
-    for (int c = 0; c < C::AKQ; ++c) tma_load_2d(q_stage + c * C::ATOM_COL, &qmap, c * 64, t * p.H + h0, q_full);
+    for (int c = 0; c < C::AKQ; ++c) tma_load_2d(q_stage + c * C::Q_ATOM, &qmap, c * 64, t * p.H + h0, q_full);
   }
 
   if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ gather producers (8 warps)
-    // Warp pw copies rows 8 pw .. 8 pw + 7 of each tile. Their 16-byte chunks
-    // are numbered row-major (CPR per row) and issued 32 per instruction, so
-    // most instructions move 512 contiguous bytes of one row.
+    // Warp pw copies rows RPW pw .. RPW pw + RPW - 1 of each tile. Their
+    // 16-byte chunks are numbered row-major (CPR per row) and issued 32 per
+    // instruction, so most instructions move 512 contiguous bytes of one row.
     pdl_wait_prior();
     constexpr int CPR = C::DP / 8;                 // 16-byte chunks per stored row
-    constexpr int ROUNDS = (8 * CPR + 31) / 32;    // instructions per warp per tile
+    constexpr int ROUNDS = (C::RPW * CPR + 31) / 32;  // instructions per warp per tile
     const int pw = warp - 4;
     const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * D;
     auto row_index = [&](int tile) -> int {
-      const int k = k_begin + tile * C::TK + 8 * pw + lane;
-      return (lane < 8 && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
+      const int k = k_begin + tile * C::TK + C::RPW * pw + lane;
+      return (lane < C::RPW && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
     };
     int nxt = row_index(0);
     bool ok = true;
@@ -243,17 +263,17 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
       if (ok) ok = mbar_wait_warp(&kv_empty[sl], (use & 1u) ^ 1u, abort_flag);
       if (!ok) break;
       const bool okr = cur >= 0 && cur < len;
-      if (lane < 8 && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
+      if (lane < C::RPW && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
       const int mine = okr ? cur : -1;
       const uint32_t stage = smem_u32(smem + C::OFF_KV + sl * C::KV_BYTES);
 #pragma unroll 2
       for (int q = 0; q < ROUNDS; ++q) {
         const int flat = q * 32 + lane;                  // chunk number within the warp's rows
-        const int rl = flat / CPR;                       // row of the warp (0..7)
+        const int rl = flat / CPR;                       // row of the warp (0..RPW-1)
         const int c = flat - rl * CPR;                   // 16-byte chunk of the row
-        const int srow = __shfl_sync(0xffffffffu, mine, rl & 7);
-        if (flat < 8 * CPR) {
-          const int r = 8 * pw + rl;
+        const int srow = __shfl_sync(0xffffffffu, mine, rl < C::RPW ? rl : 0);
+        if (flat < C::RPW * CPR) {
+          const int r = C::RPW * pw + rl;
           const bool has = srow >= 0 && c * 8 < D;
           const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * D + (has ? c * 8 : 0);
           cp_async_16(stage + (c >> 3) * C::ATOM_COL + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
@@ -283,7 +303,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         for (int nb = 0; nb < C::PV_MMAS; ++nb) {
 #pragma unroll
           for (int kk = 0; kk < C::TK / 16; ++kk) {
-            const uint64_t a = smem_desc_sw128(p_base + kk * 32, 16, 1024);
+            const uint64_t a = smem_desc_sw128(p_base + (kk >> 2) * (C::HB * 128) + (kk & 3) * 32, 16, 1024);
             // V = first DC dims of the gathered rows, MN-major: 64-dim atom columns
             // ATOM_COL bytes apart (LBO), 8-key row groups 1024 bytes apart (SBO).
             const uint64_t bd =
@@ -350,7 +370,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         uint32_t v[32];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          q_pair<C::ATOM_COL>(q_stage, ha, hbr, 64 * g + 8 * j + cc, v[4 * j], v[4 * j + 1], v[4 * j + 2],
+          q_pair<C::Q_ATOM>(q_stage, ha, hbr, 64 * g + 8 * j + cc, v[4 * j], v[4 * j + 1], v[4 * j + 2],
                               v[4 * j + 3]);
         tmem_st16x256_x8(tmem_base + lane_addr + lo16 + C::COL_Q + 64 * g, v);
       }
@@ -358,7 +378,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         uint32_t v[16];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          q_pair<C::ATOM_COL>(q_stage, ha, hbr, (QCOLS / 64) * 64 + 8 * j + cc, v[4 * j], v[4 * j + 1],
+          q_pair<C::Q_ATOM>(q_stage, ha, hbr, (QCOLS / 64) * 64 + 8 * j + cc, v[4 * j], v[4 * j + 1],
                               v[4 * j + 2], v[4 * j + 3]);
         tmem_st16x256_x4(tmem_base + lane_addr + lo16 + C::COL_Q + (QCOLS / 64) * 64, v);
       }
@@ -372,22 +392,32 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     float m_a = -INFINITY, m_b = -INFINITY;  // running max per row (log2 domain)
     float l_a = 0.0f, l_b = 0.0f;            // this thread's share of the running sums
     uint8_t* p_tile = smem + C::OFF_P;
-    // indices of the next tile (for the validity mask), one tile ahead
-    int i0n = (k_begin + lane < k_end) ? ld_dep(idx_row + k_begin + lane) : -1;
-    int i1n = (k_begin + 32 + lane < k_end) ? ld_dep(idx_row + k_begin + 32 + lane) : -1;
+    // indices of the next tile (for the validity mask), one tile ahead:
+    // lane l holds keys l, 32 + l and (80-key tiles) 64 + l of the tile
+    constexpr int REPS = C::TK / 8;   // 8-column repetitions of the 16x256b layout
+    auto idx_at = [&](int k) -> int { return k < k_end ? ld_dep(idx_row + k) : -1; };
+    int i0n = idx_at(k_begin + lane), i1n = idx_at(k_begin + 32 + lane);
+    int i2n = (C::TK > 64 && lane < C::TK - 64) ? idx_at(k_begin + 64 + lane) : -1;
     for (int it = 0; it < n_tiles && ok; ++it) {
-      const int i0 = i0n, i1 = i1n;
+      const int i0 = i0n, i1 = i1n, i2 = i2n;
       if (it + 1 < n_tiles) {
         const int kn = k_begin + (it + 1) * C::TK;
-        i0n = (kn + lane < k_end) ? ld_dep(idx_row + kn + lane) : -1;
-        i1n = (kn + 32 + lane < k_end) ? ld_dep(idx_row + kn + 32 + lane) : -1;
+        i0n = idx_at(kn + lane);
+        i1n = idx_at(kn + 32 + lane);
+        if (C::TK > 64) i2n = (lane < C::TK - 64) ? idx_at(kn + 64 + lane) : -1;
       }
       const unsigned v0 = __ballot_sync(0xffffffffu, i0 >= 0 && i0 < len);
       const unsigned v1 = __ballot_sync(0xffffffffu, i1 >= 0 && i1 < len);
+      const unsigned v2 = __ballot_sync(0xffffffffu, i2 >= 0 && i2 < len);
       if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      float v[32];
-      tmem_ld16x256_x8(tmem_base + lane_addr + lo16 + C::COL_S, v);
+      float v[4 * REPS];
+      {
+        float* v8 = v;
+        tmem_ld16x256_x8(tmem_base + lane_addr + lo16 + C::COL_S, *reinterpret_cast<float(*)[32]>(v8));
+        if constexpr (REPS > 8)
+          tmem_ld16x256_x2(tmem_base + lane_addr + lo16 + C::COL_S + 64, *reinterpret_cast<float(*)[8]>(v + 32));
+      }
       tmem_wait_ld();
       // the S buffer is free again: the next QK^T may overwrite it
       tc_fence_before();
@@ -396,11 +426,12 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
       // v[4j + 0/1] = row ra, cols 8j+cc, +1; v[4j + 2/3] = row ra+8, same cols
       float ta = -INFINITY, tb = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < REPS; ++j) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int col = 8 * j + cc + e;
-          const bool valid = (col < 32) ? ((v0 >> col) & 1u) : ((v1 >> (col - 32)) & 1u);
+          const unsigned vm = col < 32 ? v0 : col < 64 ? v1 : v2;
+          const bool valid = (vm >> (col & 31)) & 1u;
           v[4 * j + e] = valid ? v[4 * j + e] * p.scale_log2 : -INFINITY;
           v[4 * j + 2 + e] = valid ? v[4 * j + 2 + e] * p.scale_log2 : -INFINITY;
           ta = fmaxf(ta, v[4 * j + e]);
@@ -449,9 +480,9 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         tmem_wait_st();
       }
       // P = 2^(s - m) in bf16; the sums add the rounded values PV actually uses
-      uint32_t pa[8], pb[8];
+      uint32_t pa[REPS], pb[REPS];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < REPS; ++j) {
         const float a0 = (m_a == -INFINITY) ? 0.0f : ex2_approx(v[4 * j] - m_a);
         const float a1 = (m_a == -INFINITY) ? 0.0f : ex2_approx(v[4 * j + 1] - m_a);
         const float b0 = (m_b == -INFINITY) ? 0.0f : ex2_approx(v[4 * j + 2] - m_b);
@@ -467,11 +498,14 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         if (!(ok = mbar_wait_warp(o_done, (it - 1) & 1, abort_flag))) break;  // P buffer free
       }
       {
+        // P in 64-key atom columns (K-major, 128-byte swizzle): keys 8j..8j+7
+        // are chunk j % 8 of atom column j / 8
         const int ha = sw * 16 + ra, hbr = ha + 8;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(ha, j) + 2 * cc) = pa[j];
-          *reinterpret_cast<uint32_t*>(p_tile + sw128_offset(hbr, j) + 2 * cc) = pb[j];
+        for (int j = 0; j < REPS; ++j) {
+          uint8_t* atom = p_tile + (j >> 3) * (C::HB * 128);
+          *reinterpret_cast<uint32_t*>(atom + sw128_offset(ha, j & 7) + 2 * cc) = pa[j];
+          *reinterpret_cast<uint32_t*>(atom + sw128_offset(hbr, j & 7) + 2 * cc) = pb[j];
         }
       }
       fence_proxy_async_smem();
