@@ -12,6 +12,7 @@
 #include "indexer.cuh"
 #include "quant.cuh"
 #include "sparse_mla.cuh"
+#include "sparse_mla_pipe.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -184,7 +185,62 @@ size_t mla_part_bytes(int T, int hb, int splits, int dc) {
   return align256(rows * dc * sizeof(float)) + align256(rows * sizeof(float2));
 }
 
-// Upper bound over the head-block counts a call can use (1 or 2).
+// How many clusters of `size` pipeline CTAs the device holds at once (a
+// cluster must fit inside one GPC, so this is below sms / size when the GPCs
+// do not divide evenly). Queried once per size; `fallback` when the query
+// is unavailable.
+int pipe_max_clusters(int size, int fallback);
+
+// The two-CTA pipeline for 128 heads (one score CTA and one value CTA per
+// pair; the pairs of one query form one cluster of 2 x splits CTAs). The
+// time of a launch is about (waves of clusters) x (key tiles per split), so
+// take the split count, at most PipeCfg::MAX_SPLITS, that minimises that
+// product, the fewer splits on ties (less merging). `max_clusters(s)` is the
+// number of clusters of 2s CTAs resident at once.
+template <typename MaxClusters>
+MlaPlan pipe_plan_with(int T, int K, MaxClusters max_clusters) {
+  using C = PipeCfg;
+  const int tiles = (K + C::TK - 1) / C::TK;
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int sp = 1; sp <= C::MAX_SPLITS && sp <= tiles; ++sp) {
+    const int mc = max_clusters(sp);
+    if (mc < 1) break;
+    const int64_t waves = (static_cast<int64_t>(T) + mc - 1) / mc;
+    const int64_t cost = waves * ((tiles + sp - 1) / sp);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  const int tps = (tiles + best - 1) / best;
+  const int splits = (tiles + tps - 1) / tps;
+  return MlaPlan{splits, tps * C::TK};
+}
+
+MlaPlan pipe_plan(int T, int K, int sms) {
+  return pipe_plan_with(T, K, [sms](int sp) { return pipe_max_clusters(2 * sp, sms / (2 * sp)); });
+}
+
+// Workspace of the pipeline: the P rings and final row statistics (one per
+// SM a score CTA can run on), then the split partials (128 rows per pair).
+size_t pipe_ring_bytes() {
+  using C = PipeCfg;
+  return align256(static_cast<size_t>(C::RING_SMS) * C::NP * C::SLOT_BYTES) +
+         align256(static_cast<size_t>(C::RING_SMS) * C::M * sizeof(float2));
+}
+
+size_t pipe_ws_bytes(int T, int splits) {
+  size_t b = pipe_ring_bytes();
+  if (splits > 1) {
+    const size_t rows = static_cast<size_t>(T) * splits * PipeCfg::M;
+    b += align256(rows * PipeCfg::DC * sizeof(float)) + align256(rows * sizeof(float2));
+  }
+  return b;
+}
+
+// Upper bound over the kernels a call can use: the 64-head kernel with 1 or
+// 2 head blocks, and the two-CTA pipeline.
 size_t mla_ws_bytes(const dsa_batch* bt, int k) {
   const int T = bt->num_q;
   size_t need = 0;
@@ -193,7 +249,8 @@ size_t mla_ws_bytes(const dsa_batch* bt, int k) {
     const size_t b = mla_part_bytes(T, hb, pl.splits, kMlaMaxLatent);
     need = b > need ? b : need;
   }
-  return need;
+  const size_t bp = pipe_ws_bytes(T, pipe_plan(T, k, num_sms()).splits);
+  return bp > need ? bp : need;
 }
 
 // ---------------------------------------------------------------- launches
@@ -401,9 +458,103 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   return check_launch("sparse_mla");
 }
 
+int pipe_max_clusters(int size, int fallback) {
+  static std::mutex mu;
+  static int cache[2 * PipeCfg::MAX_SPLITS + 1] = {};
+  if (size < 1 || size > 2 * PipeCfg::MAX_SPLITS) return fallback;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[size] == 0) {
+    int n = 0;
+    // (no error message is recorded here: a size query may run without a device)
+    if (cudaFuncSetAttribute(sparse_mla_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             PipeCfg::SMEM_BYTES) == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(size, 1, 1);
+      cfg.blockDim = dim3(PipeCfg::THREADS);
+      cfg.dynamicSmemBytes = PipeCfg::SMEM_BYTES;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = size;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      if (cudaOccupancyMaxActiveClusters(&n, sparse_mla_pipe_kernel, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();  // clear a failed query's error state
+    cache[size] = n > 0 ? n : -1;
+  }
+  return cache[size] > 0 ? cache[size] : fallback;
+}
+
+dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
+                           float* lse, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl) {
+  using C = PipeCfg;
+  dsa_status s = set_smem(sparse_mla_pipe_kernel, C::SMEM_BYTES);
+  if (s != DSA_OK) return s;
+  const int T = bt->num_q;
+  const MlaPlan pl = pipe_plan(T, k, num_sms());
+  const size_t need = pipe_ws_bytes(T, pl.splits);
+  if (!ws || ws_bytes < need)
+    return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "attention workspace %zu < %zu bytes", ws_bytes, need);
+  if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  CUtensorMap qmap;
+  if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(T) * C::M, C::D, C::M)) != DSA_OK) return s;
+  PipeParams p;
+  p.cu_q = bt->cu_q;
+  p.seq_lens = bt->seq_lens;
+  p.B = bt->batch;
+  p.L_max = bt->max_seq_len;
+  p.T = T;
+  p.K = k;
+  p.idx = idx;
+  p.scale_log2 = in->softmax_scale * 1.4426950408889634f;
+  p.keys_per_split = pl.keys_per_split;
+  p.splits = pl.splits;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  p.ring = w;
+  w += align256(static_cast<size_t>(C::RING_SMS) * C::NP * C::SLOT_BYTES);
+  p.fin = reinterpret_cast<float2*>(w);
+  w += align256(static_cast<size_t>(C::RING_SMS) * C::M * sizeof(float2));
+  p.part_o = nullptr;
+  p.part_ml = nullptr;
+  if (pl.splits > 1) {
+    const size_t rows = static_cast<size_t>(T) * pl.splits * C::M;
+    p.part_o = reinterpret_cast<float*>(w);
+    p.part_ml = reinterpret_cast<float2*>(w + align256(rows * C::DC * sizeof(float)));
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pl.splits, T, 1);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 2 * pl.splits;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, sparse_mla_pipe_kernel, static_cast<const __nv_bfloat16*>(in->kv), qmap, p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla_pipe launch: %s", cudaGetErrorString(e));
+  return check_launch("sparse_mla_pipe");
+}
+
 dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
                       void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false) {
   const int hb = (in->n_heads + 63) / 64;
+  if (in->d_latent == 512 && in->n_heads == PipeCfg::M && bt->num_q <= 65535)  // queries on grid y
+    return launch_mla_pipe(bt, in, idx, k, out, lse, ws, ws_bytes, st, pdl);
   if (in->d_latent == 512) {
     const MlaPlan pl = mla_plan(bt->num_q, hb, k, num_sms(), MlaCfg<576, 512>::TK);
     return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);

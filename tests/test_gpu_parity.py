@@ -199,10 +199,11 @@ def _mla_check(wl, idx_np):
 
 @pytest.mark.parametrize("T_per_seq,H", [(1, 128), (16, 128), (40, 128), (1, 64), (40, 64)])
 def test_mla_matches_oracle(T_per_seq, H):
-    """128 heads (CTA pairs splitting the row dims): T_per_seq=1 -> 2 queries,
-    3 key splits merged in a cluster of 6; 16 -> 32 queries, 2 splits; 40 ->
-    80 queries, one split each. 64 heads (one CTA per head block): the same
-    split regimes. K=300 leaves a ragged 64-key tail and -1 padding."""
+    """128 heads (score CTA + value CTA pairs): T_per_seq=1 -> 2 queries, 3
+    key splits (a cluster of 6 CTAs, merged through the workspace); 16 -> 32
+    queries, split in 2; 40 -> 80 queries, one split each. 64 heads (one CTA
+    per head block): the same split regimes. K=300 leaves a ragged 64-key
+    tail and -1 padding."""
     wl = W.scaled("c2", B=2, Lmax=900, lens=(900, 400), T_per_seq=T_per_seq, K=300, H=H)
     rng = np.random.default_rng(T_per_seq)
     nv = wl.n_valid()
