@@ -371,6 +371,9 @@ dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int
   p.idx = idx;
   p.bm_words = 0;
   const int L = bt->max_seq_len;
+  // short rows: one read of the row into registers (8 or 16 keys a thread)
+  if (L <= 1024 * 8) return launch_topk_kernel(topk_reg_kernel<1024, 8>, 1024, 0, p, bt->num_q, st, pdl);
+  if (L <= 1024 * 16) return launch_topk_kernel(topk_reg_kernel<1024, 16>, 1024, 0, p, bt->num_q, st, pdl);
   // two streaming passes with position bitmaps in shared memory: the bitmaps
   // and first-digit histogram are fixed; the candidate list of the threshold
   // bin gets a quarter of a row (at least 2048, at most 16384 slots) within

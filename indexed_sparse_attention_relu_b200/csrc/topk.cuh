@@ -8,9 +8,11 @@
 //
 // Method: scores map to order-preserving uint32 keys (-0 == +0); one CTA per
 // row finds the K-th largest key tau and `need` = how many keys equal to tau
-// must be taken (the lowest positions win). topk_bitmap_kernel (every row
-// whose position bitmaps fit in shared memory) needs two streaming passes
-// over the row; topk_kernel (longer rows) one pass per 8-bit radix digit.
+// must be taken (the lowest positions win). topk_reg_kernel (rows of at most
+// 16384 positions) reads the row once into registers; topk_bitmap_kernel
+// (every row whose position bitmaps fit in shared memory) needs two
+// streaming passes over the row; topk_kernel (longer rows) one pass per
+// 8-bit radix digit.
 // Both emit the selected positions in position order with two block-wide
 // exclusive scans, so the output comes out sorted with no sort. The result
 // depends only on the scores (bit-deterministic).
@@ -207,6 +209,141 @@ __global__ void __launch_bounds__(THREADS) topk_kernel(const TopkParams p) {
 // Emission walks the bitmaps in position order with two block scans (the
 // first ranks the equal keys, the second places the outputs), so the indices
 // come out ascending with no sort.
+// Rows of at most THREADS * PER positions. Thread `tid` owns positions
+// [tid * PER, tid * PER + PER) and loads their keys once into registers. The
+// K-th largest key tau is built from four 8-bit digits, most significant
+// first; each digit is counted in per-warp histograms (no two warps share a
+// counter) among the keys that match the digits found so far, and the bin
+// holding the remaining rank is found with one scan over the 256 bins in
+// descending order. Emission: keys above tau, plus the `need` lowest-position
+// keys equal to tau, written in position order after one block scan of the
+// packed (equal, above) counts: the equal keys taken before a thread are
+// min(equal keys before it, need).
+template <int THREADS, int PER>
+__global__ void __launch_bounds__(THREADS, 1) topk_reg_kernel(const TopkParams p) {
+  static_assert(PER % 4 == 0 && PER <= 32, "whole float4 groups, one mask word");
+  static_assert(THREADS >= 256, "one thread per digit bin");
+  static_assert(THREADS * PER < 65536, "packed 16-bit counts in the emission scan");
+  constexpr int NWARP = THREADS / 32;
+  using Scan = cub::BlockScan<int, THREADS>;
+  __shared__ typename Scan::TempStorage scan_tmp;
+  __shared__ uint32_t hist[NWARP][256];
+  __shared__ int wsum[8];
+  __shared__ int s_digit, s_krem;
+
+  const int t = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int lane = lane_id();
+  const int warp = warp_id();
+  const int b = seq_of_token(p.cu_q, p.B, t);
+  const int len = min(__ldg(p.seq_lens + b), p.L_max);
+  const int n = max(0, min(__ldg(p.q_pos + t) + 1, len));
+  int32_t* out = p.idx + static_cast<int64_t>(t) * p.K;
+  const float* row = p.scores + static_cast<int64_t>(t) * p.ld;
+  pdl_launch_dependents();  // the attention may be scheduled; it waits for these indices
+  pdl_wait_prior();         // the indexer's scores (and anything before it) are complete
+
+  if (n <= p.K) {
+    for (int i = tid; i < p.K; i += THREADS) out[i] = (i < n) ? i : -1;
+    return;
+  }
+  const int base = tid * PER;
+  uint32_t key[PER];
+  uint32_t valid = 0u;
+  if (base + PER <= n && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+#pragma unroll
+    for (int c = 0; c < PER / 4; ++c) {
+      const float4 v = ld_dep4(row + base + 4 * c);
+      key[4 * c] = float_order_key(v.x);
+      key[4 * c + 1] = float_order_key(v.y);
+      key[4 * c + 2] = float_order_key(v.z);
+      key[4 * c + 3] = float_order_key(v.w);
+    }
+    valid = (PER == 32) ? ~0u : ((1u << PER) - 1u);
+  } else {
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+      key[u] = 0u;
+      if (base + u < n) {
+        key[u] = float_order_key(ld_dep(row + base + u));
+        valid |= 1u << u;
+      }
+    }
+  }
+
+  // ---- the K-th largest key, 8 bits at a time
+  uint32_t prefix = 0u, pmask = 0u;
+  int kr = p.K;  // rank of tau among the keys that match the prefix
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    uint32_t* h = hist[warp];
+#pragma unroll
+    for (int i = lane; i < 256; i += 32) h[i] = 0u;
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < PER; ++u)
+      if (((valid >> u) & 1u) && (key[u] & pmask) == prefix) atomicAdd(&h[(key[u] >> shift) & 255u], 1u);
+    __syncthreads();
+    int cnt = 0, incl = 0;
+    if (tid < 256) {
+      const int d = 255 - tid;  // descending digit order
+#pragma unroll 8
+      for (int w = 0; w < NWARP; ++w) cnt += static_cast<int>(hist[w][d]);
+      incl = cnt;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      if (lane == 31) wsum[warp] = incl;
+    }
+    __syncthreads();
+    if (tid < 256) {
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += wsum[w];
+      incl += before;
+      const int excl = incl - cnt;
+      if (excl < kr && kr <= incl) {
+        s_digit = 255 - tid;
+        s_krem = kr - excl;
+      }
+    }
+    __syncthreads();
+    kr = s_krem;
+    prefix |= static_cast<uint32_t>(s_digit) << shift;
+    pmask |= 255u << shift;
+  }
+  const uint32_t tau = prefix;
+  const int need = kr;  // keys equal to tau that are taken, lowest positions first
+
+  // ---- emission in position order
+  uint32_t selm = 0u, eqm = 0u;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    if (!((valid >> u) & 1u)) continue;
+    if (key[u] > tau) selm |= 1u << u;
+    else if (key[u] == tau) eqm |= 1u << u;
+  }
+  const int ce = __popc(eqm);
+  int packed_before;
+  Scan(scan_tmp).ExclusiveSum((ce << 16) | __popc(selm), packed_before);
+  const int eq_before = packed_before >> 16;
+  const int take = max(0, min(ce, need - eq_before));
+  int o = (packed_before & 0xffff) + min(eq_before, need);
+  int e = 0;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const bool sel = (selm >> u) & 1u;
+    const bool eq = (eqm >> u) & 1u;
+    if (sel || (eq && e < take)) {
+      if (o < p.K) out[o] = base + u;
+      ++o;
+    }
+    if (eq) ++e;
+  }
+}
+
 template <int THREADS>
 __device__ __forceinline__ void topk_find_digit(const uint32_t* h256, int width, int& kr, int* wsum, int* s_digit,
                                                 int* s_krem) {

@@ -169,6 +169,27 @@ def test_topk_tie_cases():
     assert list(idx[2][:40]) == list(range(40)) and np.all(idx[2][40:] == -1)
 
 
+def test_topk_register_rows_full_and_ragged():
+    """Rows held in registers: 8192 positions (8 keys a thread, aligned
+    vector loads, the decode shape with K = 2048) and up to 16383 positions
+    (16 keys a thread; an odd row stride leaves rows unaligned, so keys load
+    one at a time), with ties at the threshold and an all-equal row."""
+    rng = np.random.default_rng(11)
+    full = [W.bf16_round(rng.standard_normal(8192).astype(np.float32) * 8),
+            np.float32(rng.integers(-20, 20, 8192)),
+            np.zeros(8192, np.float32)]
+    idx, sc, lens = _topk_rows(full, 2048)
+    assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
+    assert list(idx[2]) == list(range(2048))
+    ragged = [W.bf16_round(rng.standard_normal(16383).astype(np.float32) * 8),
+              np.float32(rng.integers(-20, 20, 12001)),
+              np.zeros(9000, np.float32),
+              W.bf16_round(rng.standard_normal(2049).astype(np.float32)),
+              np.float32(rng.integers(0, 3, 1500))]
+    idx, sc, lens = _topk_rows(ragged, 2048)
+    assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
+
+
 def test_topk_long_rows_and_crowded_threshold_bin():
     """Long rows (two streaming passes), and rows whose threshold bin holds more
     keys than the candidate list (all equal, or a constant bulk under a few
