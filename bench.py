@@ -135,9 +135,10 @@ class ClockSampler:
                 "power_w_max": max(p for _, p, _ in self.samples)}
 
 
-def run_cpu_oracle(wl, n_tokens: int, seed: int = 0):
+def run_cpu_oracle(wl, n_tokens: int, seed: int = 0, min_seconds: float = 0.0):
     """Time the fp64 oracle (indexer + Top-K + attention) on n_tokens sampled
-    query tokens of the workload. Returns (tokens, seconds, threads)."""
+    query tokens of the workload, repeated until at least min_seconds of CPU
+    work have been timed. Returns (tokens processed, seconds, threads)."""
     import oracle
     from indexed_sparse_attention_relu_b200 import workloads as W
     rng = np.random.default_rng(seed)
@@ -147,10 +148,13 @@ def run_cpu_oracle(wl, n_tokens: int, seed: int = 0):
     if wl.key_dtype == "fp8":
         codes, scales = oracle.quantize_keys(sub.k_idx, sub.scale_group)
         kw = dict(k_codes=codes, k_scales=scales)
-    t0 = time.perf_counter()
-    oracle.dsa(sub, **kw)
-    dt = time.perf_counter() - t0
-    return len(rows), dt, oracle.num_threads()
+    done, dt = 0, 0.0
+    while done == 0 or dt < min_seconds:
+        t0 = time.perf_counter()
+        oracle.dsa(sub, **kw)
+        dt += time.perf_counter() - t0
+        done += len(rows)
+    return done, dt, oracle.num_threads()
 
 
 def reference_arm(args, rank: int):
@@ -190,6 +194,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--copies", type=int, default=4, help="rotating input copies (L2 defeat)")
     ap.add_argument("--cpu-tokens", type=int, default=8, help="query tokens in the oracle baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="minimum CPU time of the oracle baseline")
     ap.add_argument("--ref-tokens", type=int, default=1, help="query tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph")
@@ -389,10 +394,10 @@ def main():
         "device_status": [status, status2],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, dt, thr = run_cpu_oracle(wl, args.cpu_tokens)
+        n, dt, thr = run_cpu_oracle(wl, args.cpu_tokens, min_seconds=args.cpu_seconds)
         line["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
-                                "sample": f"{n} query tokens of the same workload (full causal history), fp64, "
-                                          f"{dt:.1f} s"}
+                                "sample": f"{min(args.cpu_tokens, wl.T)} query tokens of the same workload (full "
+                                          f"causal history), fp64, repeated to {n} tokens in {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
