@@ -366,11 +366,12 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
 #pragma unroll
           for (int q = 0; q < 4; ++q) tmem_ld16(tmem_base + lane_addr + acc * C::N + c + 16 * q, v[q]);
           tmem_wait_ld();
-          float tok = 0.0f;
+          float t4[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // four partial sums (short dependency chains)
 #pragma unroll
           for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int u = 0; u < 16; ++u) tok = fmaf(w_s[c + 16 * q + u], fmaxf(v[q][u], 0.0f), tok);
+            for (int u = 0; u < 16; ++u) t4[u & 3] = fmaf(w_s[c + 16 * q + u], fmaxf(v[q][u], 0.0f), t4[u & 3]);
+          const float tok = (t4[0] + t4[1]) + (t4[2] + t4[3]);
           const int g = c / HI;
 #pragma unroll
           for (int gg = 0; gg < G; ++gg)
@@ -384,9 +385,10 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
           float v[16];
           tmem_ld16(tmem_base + lane_addr + acc * C::N + c, v);
           tmem_wait_ld();
-          float chunk = 0.0f;
+          float t4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-          for (int u = 0; u < 16; ++u) chunk = fmaf(w_s[c + u], fmaxf(v[u], 0.0f), chunk);
+          for (int u = 0; u < 16; ++u) t4[u & 3] = fmaf(w_s[c + u], fmaxf(v[u], 0.0f), t4[u & 3]);
+          const float chunk = (t4[0] + t4[1]) + (t4[2] + t4[3]);
           const int g = c / HI;
 #pragma unroll
           for (int gg = 0; gg < G; ++gg)
