@@ -418,10 +418,31 @@ __global__ void __launch_bounds__(THREADS, 1) topk_bitmap_kernel(const TopkParam
   if (tid == 0) s_ncand = 0;
   __syncthreads();
 
-  // ---- A: first-digit histogram (four independent loads in flight per thread)
+  // ---- A: first-digit histogram (four 16-byte loads in flight per thread on
+  // aligned rows: the streaming passes are bound by loads in flight)
   {
     uint32_t* myh = hist + (warp & (HCOPIES - 1)) * NB;
-    for (int i0 = tid; i0 < n; i0 += 4 * THREADS) {
+    int done = 0;
+    if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+      const int n4 = n >> 2;  // whole groups of four positions
+      for (int g0 = tid; g0 < n4; g0 += 4 * THREADS) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          v[u] = (g0 + u * THREADS < n4) ? ld_dep4(row + 4 * (g0 + u * THREADS)) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (g0 + u * THREADS < n4) {
+            atomicAdd(&myh[float_order_key(v[u].x) >> LOW], 1u);
+            atomicAdd(&myh[float_order_key(v[u].y) >> LOW], 1u);
+            atomicAdd(&myh[float_order_key(v[u].z) >> LOW], 1u);
+            atomicAdd(&myh[float_order_key(v[u].w) >> LOW], 1u);
+          }
+        }
+      }
+      done = 4 * n4;
+    }
+    for (int i0 = done + tid; i0 < n; i0 += 4 * THREADS) {
       float v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) v[u] = (i0 + u * THREADS < n) ? ld_dep(row + i0 + u * THREADS) : 0.0f;
@@ -456,21 +477,33 @@ __global__ void __launch_bounds__(THREADS, 1) topk_bitmap_kernel(const TopkParam
   int kr = p.K - s_above;  // keys to take from bin b*
 
   // ---- B: positions in higher bins -> selection bitmap; keys in b* -> candidates
-  for (int i0 = warp * 32; i0 < n; i0 += THREADS) {
-    const int i = i0 + lane;
-    const bool valid = i < n;
-    const uint32_t key = valid ? float_order_key(ld_dep(row + i)) : 0u;
-    const uint32_t kb = key >> LOW;
-    const unsigned selmask = __ballot_sync(0xffffffffu, valid && kb > bstar);
-    if (lane == 0 && selmask) selb[i0 >> 5] = selmask;
-    const unsigned cmask = __ballot_sync(0xffffffffu, valid && kb == bstar);
-    if (cmask) {
-      int base = 0;
-      if (lane == 0) base = atomicAdd(&s_ncand, __popc(cmask));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if ((cmask >> lane) & 1u) {
-        const int slot = base + __popc(cmask & ((1u << lane) - 1u));
-        if (slot < p.cache_cap) cands[slot] = make_uint2(key, static_cast<uint32_t>(i));
+  // (a warp covers 32 consecutive positions per chunk; four chunks' loads in flight)
+  for (int i00 = warp * 32; i00 < n; i00 += 4 * THREADS) {
+    float x[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i = i00 + k * THREADS + lane;
+      x[k] = (i < n) ? ld_dep(row + i) : 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int i0 = i00 + k * THREADS;  // warp-uniform
+      if (i0 >= n) break;
+      const int i = i0 + lane;
+      const bool valid = i < n;
+      const uint32_t key = valid ? float_order_key(x[k]) : 0u;
+      const uint32_t kb = key >> LOW;
+      const unsigned selmask = __ballot_sync(0xffffffffu, valid && kb > bstar);
+      if (lane == 0 && selmask) selb[i0 >> 5] = selmask;
+      const unsigned cmask = __ballot_sync(0xffffffffu, valid && kb == bstar);
+      if (cmask) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&s_ncand, __popc(cmask));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if ((cmask >> lane) & 1u) {
+          const int slot = base + __popc(cmask & ((1u << lane) - 1u));
+          if (slot < p.cache_cap) cands[slot] = make_uint2(key, static_cast<uint32_t>(i));
+        }
       }
     }
   }

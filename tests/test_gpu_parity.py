@@ -190,6 +190,19 @@ def test_topk_register_rows_full_and_ragged():
     assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
 
 
+def test_topk_streaming_rows_unaligned():
+    """Rows above 16384 positions stream from memory; an odd row stride leaves
+    all but the first row unaligned (positions load one at a time) and the
+    lengths leave ragged ends after the last whole group of four."""
+    rng = np.random.default_rng(13)
+    rows = [W.bf16_round(rng.standard_normal(20001).astype(np.float32) * 8),
+            W.bf16_round(rng.standard_normal(17003).astype(np.float32) * 8),
+            np.float32(rng.integers(-30, 30, 18002)),
+            W.bf16_round(rng.standard_normal(16385).astype(np.float32))]
+    idx, sc, lens = _topk_rows(rows, 2048)
+    assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
+
+
 def test_topk_long_rows_and_crowded_threshold_bin():
     """Long rows (two streaming passes), and rows whose threshold bin holds more
     keys than the candidate list (all equal, or a constant bulk under a few
