@@ -162,13 +162,18 @@ dsa_status dsa_topk(const dsa_batch *batch, const float *scores, int64_t score_l
  * lse: fp32 [T, n_heads] natural-log sum-exp of the scaled logits, or NULL.
  * A row with no valid index gets out = 0 and lse = -inf.
  * ws: at least dsa_workspace_size(DSA_OP_SPARSE_MLA, ...) bytes, 16-byte
- *   aligned (the size is 0, and ws may be NULL, when the batch has enough
- *   queries to fill the GPU without splitting their keys).
- * Work split: one CTA per (query, 64-head block, key split). The key splits
- * of a query form a thread-block cluster; each leaves its unnormalised
- * output rows and (max, sum) statistics in ws and, after the cluster
- * barrier, the split that owns a head merges it. DSA_ERR_WORKSPACE_TOO_SMALL
- * if ws is smaller than that call needs. */
+ *   aligned, owned by the caller and not kept after the call's kernels end.
+ *   The size is an upper bound over the head counts a call may use (the
+ *   query does not take n_heads); it includes about 17.6 MB of P rings for
+ *   128-head calls. A call that needs less may pass less.
+ * Work split. 128 heads with d_latent = 512: a pair of CTAs per (query, key
+ *   split): a score CTA computes Q K^T for all heads and the softmax and
+ *   hands P to a value CTA (which holds O) through a per-SM ring in ws.
+ *   Other shapes: one CTA per (query, 64-head block, key split). In both,
+ *   the key splits of a query form a thread-block cluster; each leaves its
+ *   unnormalised output rows and (max, sum) statistics in ws and, after the
+ *   cluster barrier, the rows are merged with a running maximum.
+ * DSA_ERR_WORKSPACE_TOO_SMALL if ws is smaller than that call needs. */
 dsa_status dsa_sparse_mla_attn(const dsa_batch *batch, const dsa_mla_in *in, const int32_t *idx,
                                int32_t k, void *out, float *lse, void *ws, size_t ws_bytes,
                                dsa_stream_t stream);

@@ -143,3 +143,20 @@ def test_workspace_sizes(lib):
     mla = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128)
     assert fused == 32 * 8192 * 4 + 32 * 2048 * 4 + mla
     assert lib.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, None, 2048, 64, 128) == 0
+
+
+def test_attention_workspace_layout(lib):
+    """The 128-head attention's workspace: four P slots (128 x 64 bf16 image +
+    128 fp32 factors = 16896 B) and 128 (max, sum) pairs for each of 256 SM
+    records, then, with S > 1 key splits, S x T x 128 partial rows of 512 fp32
+    plus their (max, sum). The split count comes from the device's resident
+    cluster count (or the SM count without a device): 1 to 4."""
+    b = _batch(num_q=32, batch=32, max_seq_len=8192)
+    mla = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128)
+    ring_fin = 256 * 4 * 16896 + 256 * 128 * 8
+    per_split = 32 * 128 * (512 * 4 + 8)
+    assert mla - ring_fin in (0, 2 * per_split, 3 * per_split, 4 * per_split)
+    # one query: every split count up to 4 fits in one wave; 32 key tiles -> 4 splits
+    b1 = _batch(num_q=1, batch=1, max_seq_len=8192)
+    one = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b1), 2048, 64, 128)
+    assert one == ring_fin + 4 * 128 * (512 * 4 + 8)
