@@ -284,6 +284,10 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   int tpc = (max_tiles + per_group - 1) / per_group;
   if (tpc < 2) tpc = 2;
   if (tpc > 64) tpc = 64;
+  // Single-token groups (decode): at most 16 tiles per CTA, so a ragged batch
+  // (most sequences shorter than the longest, whose length sets max_tiles)
+  // spreads its work over many short CTAs that the scheduler balances.
+  if (G == 1 && tpc > 16) tpc = 16;
   const int gy = (max_tiles + tpc - 1) / tpc;
   IndexerParams p;
   p.cu_q = bt->cu_q;
