@@ -70,7 +70,8 @@ typedef enum {
     DSA_ERR_DEVICE_INDEX = 5,       /* device status: an index out of range was skipped */
     DSA_ERR_DEVICE_TIMEOUT = 6,     /* device status: a bounded wait gave up */
     DSA_ERR_MISALIGNED = 7,         /* a pointer is not 16-byte aligned */
-    DSA_ERR_DEVICE_LAYOUT = 8       /* device status: a kernel found its shared memory misaligned */
+    DSA_ERR_DEVICE_LAYOUT = 8       /* device status: a kernel found its shared memory misaligned,
+                                       or an SM id outside its per-SM workspace records */
 } dsa_status;
 
 typedef enum { DSA_KEY_BF16 = 0, DSA_KEY_FP8_E4M3 = 1 } dsa_key_dtype;
