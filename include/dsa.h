@@ -14,19 +14,19 @@
  *   3. Sparse Flash Attention over multi-head latent attention (MLA) rows:
  *      every query head attends only over the selected latent KV rows; a row
  *      has d_latent + d_rope dims, the value is its first d_latent dims.
- * The "pseudocode: fused execution of the sparse attention path" of
  * "Inference Adaptation and Performance Optimization for New Large Language
- * Model Architectures" (section 6) splits the path as
- *   indices = lightning_indexer(query, key_cache)
- *   output  = sparse_flash_attention(query, indices, key_cache, value_cache)
- * which the calls below follow: dsa_indexer_scores + dsa_topk form the
- * indexer, dsa_sparse_mla_attn the attention, dsa_fused_decode the whole
- * chain. The index-key cache can be BF16 or FP8 E4M3 with a per-group fp32
- * scale (Tiered Quantization of "Day-0 Inference Adaptation and Performance
- * Optimization for New-Architecture Large Language Models"); both paths have
- * the same interface ("the quantized path maintains the same interface
- * semantics as the high-precision path", Layered Quantization of "Inference
- * Optimization for New Open-Source LLM Architectures ...").
+ * Model Architectures" (section 6, fused execution of the sparse attention
+ * path) splits the path into an indexer step that turns the query and the
+ * index-key cache into selected positions, and an attention step that reads
+ * only those cache rows. The calls below follow that split:
+ * dsa_indexer_scores + dsa_topk form the indexer, dsa_sparse_mla_attn the
+ * attention, dsa_fused_decode the whole chain. The index-key cache can be
+ * BF16 or FP8 E4M3 with a per-group fp32 scale (Tiered Quantization of
+ * "Day-0 Inference Adaptation and Performance Optimization for
+ * New-Architecture Large Language Models"); both key types go through the
+ * same calls with the same meaning, so a caller switches precision by the
+ * key_dtype field alone (Layered Quantization of "Inference Optimization for
+ * New Open-Source LLM Architectures").
  *
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers unless stated, row-major, owned
@@ -41,11 +41,12 @@
  *    [0, seq_len), or a bounded wait inside a kernel that gave up) never trap:
  *    the offending element is skipped and a sticky per-device status word is
  *    set; read it with dsa_read_device_status().
- *  - Supported shapes: indexer heads H_I in [1, 64] with H_I * (tokens per
- *    group) <= 256, indexer dim d_I in {32, 64, 128}; MLA (d_latent, d_rope)
- *    in {(512, 64), (64, 16)}; MLA heads H in [1, 128] (a multiple of 64 or
- *    smaller than 64); 1 <= K <= 2048. Others return
- *    DSA_ERR_UNSUPPORTED_SHAPE.
+ *  - Supported shapes (anything else returns DSA_ERR_UNSUPPORTED_SHAPE):
+ *      indexer (H_I, d_I): (4, 32), (4, 128), (64, 32), (64, 128)
+ *      MLA (d_latent, d_rope): (512, 64), (64, 16)
+ *      MLA heads H: 1..64, or 128
+ *      top-K k: 1..2048
+ *    FP8 index keys need scale_group == d_I (one scale per key).
  *  - Alignment: every tensor pointer must be 16-byte aligned.
  */
 #ifndef DSA_H_
@@ -148,7 +149,10 @@ typedef struct {
 dsa_status dsa_indexer_scores(const dsa_batch *batch, const dsa_indexer_in *in, float *scores,
                               int64_t score_ld, void *ws, size_t ws_bytes, dsa_stream_t stream);
 
-/* Per-row Top-K of the indexer scores.
+/* Per-row Top-K of the indexer scores: the selection step that ends the
+ * Lightning Indexer ("Day-0 Inference Optimization for a New Sparse
+ * Attention Architecture", section 1: only the Top-K history positions of a
+ * query are passed on to the attention).
  * scores: fp32 [T, score_ld]; only columns [0, n_valid(t)) are read.
  * idx: int32 [T, k]: the min(k, n_valid(t)) best positions of row t under the
  *   order (score desc, position asc) with -0 == +0, written in ascending
@@ -205,7 +209,9 @@ dsa_status dsa_fused_decode(const dsa_batch *batch, const dsa_indexer_in *idx_in
  * The attention runs with one key split per query, so results agree with
  * dsa_fused_decode within rounding (indices are identical).
  * The first call on a device looks up the array's device address with that
- * device current; make that first call before any stream capture.
+ * device current, and so does the first call after the device's context has
+ * changed (e.g. after cudaDeviceReset); make such a call before any stream
+ * capture.
  * All calls share the array: calls whose work overlaps on the GPU (other
  * streams, other threads) race on it and must be serialised by the caller.
  * Nothing in the array needs to start at zero; stale contents are never read. */
@@ -213,7 +219,12 @@ dsa_status dsa_fused_decode_noalloc(const dsa_batch *batch, const dsa_indexer_in
                                     const dsa_mla_in *mla_in, int32_t k, void *out, float *lse,
                                     int32_t *idx_out, dsa_stream_t stream);
 
-/* Index-key cache write: per-group dynamic FP8 quantisation.
+/* Index-key cache write: per-group dynamic FP8 quantisation, the scheme of
+ * the Tiered Quantization table of "Day-0 Inference Adaptation and
+ * Performance Optimization for New-Architecture Large Language Models"
+ * (indexer keys in 8-bit floating point, one scale per group of elements
+ * computed from the group's absolute maximum) and of its block-wise
+ * quantisation example.
  * k_bf16: bf16 [n_keys, dim]; for every group of `group` elements
  *   scale = fl32(max|k| / 448); scale == 0 -> codes 0;
  *   else code = e4m3 round-to-nearest-even, saturating, of fl32(k / scale).
@@ -222,7 +233,9 @@ dsa_status dsa_fused_decode_noalloc(const dsa_batch *batch, const dsa_indexer_in
 dsa_status dsa_quantize_index_keys(const void *k_bf16, int64_t n_keys, int32_t dim, int32_t group,
                                    uint8_t *k8, float *scale, dsa_stream_t stream);
 
-/* Dequantisation: out = fl32(decode(code) * scale), fp32 [n_keys, dim]. */
+/* Inverse of the cache write above (same passage): the value a key's FP8
+ * code stands for, out = fl32(decode(code) * scale), fp32 [n_keys, dim].
+ * Same group and dim rules as dsa_quantize_index_keys. */
 dsa_status dsa_dequantize_index_keys(const uint8_t *k8, const float *scale, int64_t n_keys,
                                      int32_t dim, int32_t group, float *out, dsa_stream_t stream);
 
@@ -234,6 +247,21 @@ size_t dsa_workspace_size(int op, const dsa_batch *batch, int32_t k, int32_t h_i
 /* Waits for `stream`, then returns in *code_out the sticky device status
  * (DSA_OK or a DSA_ERR_DEVICE_* code) of the current device and clears it. */
 dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t *code_out);
+
+/* Test hooks for the failure-detection path (not for production use; both
+ * act on the current device and are synchronous with respect to the host).
+ * dsa_debug_set_wait_limit: wall-time limit in ns of every bounded wait
+ *   inside the kernels (0 restores the default of 2 s). A shorter limit lets
+ *   a test make a wait run out quickly; it must stay far above the longest
+ *   legal wait of the calls the test makes.
+ * dsa_debug_withhold_signal: on != 0 makes the 128-head attention's score
+ *   CTA hold back its first "P ready" signal to the value CTA, so the value
+ *   CTA's wait for it runs out: the kernel records DSA_ERR_DEVICE_TIMEOUT in
+ *   the device status word, every role leaves its loop, tensor memory is
+ *   released and the kernel returns (the call's outputs are then undefined).
+ *   on = 0 restores normal operation. */
+dsa_status dsa_debug_set_wait_limit(uint64_t limit_ns);
+dsa_status dsa_debug_withhold_signal(int32_t on);
 
 /* Text for a status code (static storage). */
 const char *dsa_status_string(dsa_status s);

@@ -44,6 +44,7 @@ EXPORTED = (
     "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_fused_decode", "dsa_fused_decode_noalloc",
     "dsa_quantize_index_keys", "dsa_dequantize_index_keys", "dsa_workspace_size",
     "dsa_read_device_status", "dsa_status_string", "dsa_last_error", "dsa_version",
+    "dsa_debug_set_wait_limit", "dsa_debug_withhold_signal",
 )
 
 
@@ -96,6 +97,8 @@ def load() -> ctypes.CDLL:
             "dsa_status_string": (c_char_p, [c_int]),
             "dsa_last_error": (c_char_p, []),
             "dsa_version": (c_char_p, []),
+            "dsa_debug_set_wait_limit": (c_int, [ctypes.c_uint64]),
+            "dsa_debug_withhold_signal": (c_int, [c_int32]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -231,3 +234,13 @@ def dsa_read_device_status(stream=None) -> int:
     code = c_int32(0)
     _check(load().dsa_read_device_status(_stream(stream), ctypes.byref(code)))
     return int(code.value)
+
+
+def dsa_debug_set_wait_limit(limit_ns: int) -> None:
+    """Test hook: wall-time limit of the kernels' bounded waits (0 = default 2 s)."""
+    _check(load().dsa_debug_set_wait_limit(int(limit_ns)))
+
+
+def dsa_debug_withhold_signal(on: bool) -> None:
+    """Test hook: the 128-head attention withholds its first P-ready signal."""
+    _check(load().dsa_debug_withhold_signal(1 if on else 0))

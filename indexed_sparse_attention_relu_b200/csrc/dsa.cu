@@ -160,8 +160,9 @@ struct MlaPlan {
 };
 
 // Key splits per (token, head block): enough CTAs to fill the SMs in one
-// wave, at most 8 (the splits of one (token, head block) form a cluster and
-// merge through distributed shared memory).
+// wave, at most 8 (the splits of one (token, head block) form a cluster; each
+// leaves its partial rows in the workspace, in L2, and they merge after the
+// cluster barrier).
 MlaPlan mla_plan(int T, int HB, int K, int sms, int tk = 64) {
   const int tiles = (K + tk - 1) / tk;
   const int base = T * HB;
@@ -587,7 +588,8 @@ const char* dsa_status_string(dsa_status s) {
     case DSA_ERR_DEVICE_INDEX: return "device: out-of-range index skipped";
     case DSA_ERR_DEVICE_TIMEOUT: return "device: bounded wait gave up";
     case DSA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
-    case DSA_ERR_DEVICE_LAYOUT: return "device: shared memory window misaligned";
+    case DSA_ERR_DEVICE_LAYOUT:
+      return "device: shared memory window misaligned, or an SM id outside the per-SM workspace records";
   }
   return "unknown status";
 }
@@ -753,6 +755,20 @@ dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t* code_out) {
   return DSA_OK;
 }
 
+dsa_status dsa_debug_set_wait_limit(uint64_t limit_ns) {
+  const uint64_t v = limit_ns ? limit_ns : dsa::kDefaultWaitLimitNs;
+  const cudaError_t e = cudaMemcpyToSymbol(dsa::g_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "setting the wait limit: %s", cudaGetErrorString(e));
+  return DSA_OK;
+}
+
+dsa_status dsa_debug_withhold_signal(int32_t on) {
+  const int v = on ? 1 : 0;
+  const cudaError_t e = cudaMemcpyToSymbol(dsa::g_debug_withhold, &v, sizeof(v));
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "setting the test hook: %s", cudaGetErrorString(e));
+  return DSA_OK;
+}
+
 }  // extern "C"
 
 // ============================================================================ allocation-free variant
@@ -784,22 +800,54 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes]
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
+unsigned long long g_noalloc_ctx[kMaxDevices] = {};  // context the address belongs to
+
+// Unique id of the calling thread's current CUDA context (0 if unavailable).
+// Ids are never reused, so a reset device (a new primary context, the module
+// loaded again, possibly at another address) is told apart from the old one.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = []() -> GetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<GetCurrentFn>(p);
+  }();
+  static GetIdFn get_id = []() -> GetIdFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<GetIdFn>(p);
+  }();
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // Device address of the scratch array on the current device. The host-side
-// symbol is only a stand-in, so the address is looked up once per device
-// (with that device current) and cached.
+// symbol is only a stand-in, so the address is looked up with that device
+// current (on the first call there, and again whenever the device's context
+// has changed, e.g. after cudaDeviceReset) and cached.
 dsa_status noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_CUDA, "device ordinal %d out of range", dev);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  const unsigned long long ctx = current_context_id();  // 0: no context bound to this thread yet
+  if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // binds the device's context if needed
     if (e != cudaSuccess || !p)
       return fail(DSA_ERR_CUDA, "cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = current_context_id();
   }
   *out = g_noalloc_ptr[dev];
   return DSA_OK;

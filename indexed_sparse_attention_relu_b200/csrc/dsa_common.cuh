@@ -4,7 +4,7 @@
 // gathers, the UMMA shared-memory / instruction descriptors, and the sticky
 // device status word.
 //
-// Every wait in this library is bounded: after kWaitLimitNs of wall time a
+// Every wait in this library is bounded: after g_wait_limit_ns of wall time a
 // wait records DSA_ERR_DEVICE_TIMEOUT in the status word and returns false;
 // the caller then stops its loop and reaches the kernel's teardown (TMEM is
 // always released). Nothing here traps.
@@ -29,7 +29,20 @@ __device__ __forceinline__ void set_device_status(int code) {
   atomicCAS(&g_device_status, 0, code);
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legal wait
+// Wall-time limit of every bounded wait, in ns. 2 s is far above any legal
+// wait; dsa_debug_set_wait_limit() lowers it so a test can make a wait run
+// out in milliseconds.
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+__device__ uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
+
+// Test hook: non-zero makes the two-CTA attention's score CTA withhold its
+// first "P ready" signal, so the value CTA's bounded wait for it runs out
+// (set by dsa_debug_withhold_signal(); 0 in normal operation).
+__device__ int g_debug_withhold = 0;
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+  return *reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -88,16 +101,17 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Bounded: returns
-// false (and records a timeout) after kWaitLimitNs, or as soon as *abort is
+// false (and records a timeout) after g_wait_limit_ns, or as soon as *abort is
 // set by another role that already gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try(a, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = wait_limit_ns();
   while (true) {
     if (mbar_try(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       set_device_status(DSA_ERR_DEVICE_TIMEOUT);
       *abort = 1;
       return false;
@@ -186,10 +200,11 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   const uint32_t a = smem_u32(bar);
   if (mbar_try_cluster(a, parity)) return true;
   const uint64_t t0 = globaltimer();
+  const uint64_t limit = wait_limit_ns();
   while (true) {
     if (mbar_try_cluster(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       set_device_status(DSA_ERR_DEVICE_TIMEOUT);
       *abort = 1;
       return false;
@@ -197,30 +212,22 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_cluster_v2(uint32_t addr, float a, float b) {
-  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(a), "f"(b) : "memory");
-}
-
-__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
-               : "memory");
-  return v;
-}
-
-// Named barrier `id` (1..15) over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ---------------------------------------------------------------- proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- bulk copies
+// `bytes` (a multiple of 16) from global `src` to shared `dst` (both 16-byte
+// aligned) through the async proxy; completes as bytes on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // ---------------------------------------------------------------- cp.async
@@ -242,17 +249,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
-
-// Four rows (y0..y3) x one box of columns starting at x, written as four
-// consecutive box rows at dst (the map's swizzle applies).
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y0, int32_t y1,
-                                            int32_t y2, int32_t y3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -381,12 +377,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// Brings `bytes` (a multiple of 16) starting at `src` into L2 without using
-// shared memory; no completion is tracked.
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // Sequence of token t from cu_q[0..B]: one warp, 32 boundaries per round

@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
           t0 = globaltimer();
         } else if (*abort_flag) {
           ok = false;
-        } else if (globaltimer() - t0 > kWaitLimitNs) {
+        } else if (globaltimer() - t0 > wait_limit_ns()) {
           set_device_status(DSA_ERR_DEVICE_TIMEOUT);
           *abort_flag = 1;
           ok = false;

@@ -68,9 +68,14 @@ struct PipeCfg {
   static constexpr int NP = 4;                          // ring slots per pair
   static constexpr uint32_t COL_S = 0;                  // score CTA: S double buffer, 2 x 64 columns
   static constexpr uint32_t COL_Q = 128;                // score CTA: Q, 288 columns of bf16 pairs
-  // 0-3 softmax / rescale + epilogue, 4-11 gather, 12 MMA, 13 ring signalling (score CTA) or P copy
-  // (value CTA). 14 warps cost no registers over 13: either puts four warps on one SMSP.
-  static constexpr int NUM_WARPS = 14;
+  // 0-3 softmax / rescale, 4-11 gather, 12 MMA, 13 ring signalling (score CTA) or P copy (value
+  // CTA); the epilogue runs on warps 0-11 (three per TMEM sub-partition).
+  static constexpr int NGATHER = 8;
+  static constexpr int ROWS_PER_GW = TK / NGATHER;          // rows of a tile per gather warp
+  static constexpr int MMA_WARP = 4 + NGATHER;
+  static constexpr int AUX_WARP = MMA_WARP + 1;
+  static constexpr int EPI_WARPS = 4 + NGATHER;
+  static constexpr int NUM_WARPS = AUX_WARP + 1;
   static constexpr int THREADS = NUM_WARPS * 32;
   static constexpr int MAX_SPLITS = 4;
   // score CTA shared memory
@@ -141,7 +146,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
   if (threadIdx.x == 0) {
     if (score_cta) {
       for (int i = 0; i < C::NKS; ++i) {
-        mbar_init(&bars[i], 8 * 32);  // one asynchronous arrival per gather thread
+        mbar_init(&bars[i], C::NGATHER * 32);  // one asynchronous arrival per gather thread
         mbar_init(&bars[3 + i], 1);
       }
       mbar_init(&bars[6], 1);
@@ -158,7 +163,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       mbar_init(&bars[21], 128);
     } else {
       for (int i = 0; i < C::NVS; ++i) {
-        mbar_init(&bars[i], 8 * 32);
+        mbar_init(&bars[i], C::NGATHER * 32);
         mbar_init(&bars[3 + i], 1);
       }
       for (int i = 0; i < C::NPS; ++i) {
@@ -179,7 +184,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     fence_mbar_init();
     if (score_cta) prefetch_tensormap(&qmap);
   }
-  if (warp == 12) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(reinterpret_cast<uint32_t*>(misc), 512);
     tmem_relinquish();
   }
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     uint64_t* p_written = bars + 17;
     uint64_t* fin_written = bars + 21;
     const uint32_t q_stage = smem_u32(smem + C::A_OFF_K + C::K_BYTES);  // stages 1 and 2 hold Q first
-    if (warp == 12 && lane == 0) {
+    if (warp == C::MMA_WARP && lane == 0) {
       // the query block is an input of the call: load it now (9 atom columns of 128 rows)
       mbar_arrive_expect_tx(q_full, 9 * C::Q_ATOM);
 #pragma unroll
@@ -337,7 +342,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       // final statistics of every row, published the same way
       if (ok) fin[h] = make_float2(m, l);
       mbar_arrive(fin_written);
-    } else if (warp == 13) {
+    } else if (warp == C::AUX_WARP) {
       // ---------------------------------------------------------- ring signalling
       // Waits until all 128 softmax threads have stored tile j's P and factors,
       // then releases them to the value CTA at cluster scope. Only this warp
@@ -346,22 +351,26 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         const uint32_t p_ready_peer = mapa_shared(smem_u32(smem + C::B_OFF_BAR + 12 * 8), partner);
         const uint32_t fin_peer = mapa_shared(smem_u32(smem + C::B_OFF_BAR + 21 * 8), partner);
         bool ok = true;
+        // (test hook: a set g_debug_withhold holds back the signal of tile 0,
+        // so the value CTA's bounded wait for it runs out)
+        const bool withhold = *reinterpret_cast<volatile int*>(&g_debug_withhold) != 0;
         for (int j = 0; j < n_tiles && ok; ++j) {
           ok = mbar_wait(&p_written[j % C::NP], (j / C::NP) & 1, abort_flag);
-          if (ok) mbar_arrive_remote(p_ready_peer + (j % C::NP) * 8);
+          if (ok && !(withhold && j == 0)) mbar_arrive_remote(p_ready_peer + (j % C::NP) * 8);
         }
         if (ok && mbar_wait(fin_written, 0, abort_flag)) mbar_arrive_remote(fin_peer);
       }
       __syncwarp();
-    } else if (warp < 12) {
-      // ---------------------------------------------------------- gather whole rows (8 warps)
+    } else if (warp < C::MMA_WARP) {
+      // ---------------------------------------------------------- gather whole rows
       pdl_wait_prior();
       constexpr int CPR = C::D / 8;  // 72 chunks per row
+      constexpr int RW = C::ROWS_PER_GW;
       const int pw = warp - 4;
       const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * C::D;
       auto row_index = [&](int tile) -> int {
-        const int k = k_begin + tile * C::TK + 8 * pw + lane;
-        return (lane < 8 && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
+        const int k = k_begin + tile * C::TK + RW * pw + lane;
+        return (lane < RW && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
       };
       int nxt = row_index(0);
       bool ok = true;
@@ -373,16 +382,16 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         if (ok) ok = mbar_wait_warp(&kv_empty[sl], ((j / C::NKS) & 1) ^ 1u, abort_flag);
         if (!ok) break;
         const bool okr = cur >= 0 && cur < len;
-        if (lane < 8 && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
+        if (lane < RW && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
         const int mine = okr ? cur : -1;
         const uint32_t stage = smem_u32(smem + C::A_OFF_K + sl * C::K_BYTES);
-#pragma unroll 6
-        for (int q = 0; q < 18; ++q) {
+#pragma unroll 9
+        for (int q = 0; q < RW * CPR / 32; ++q) {
           const int flat = q * 32 + lane;
           const int rl = flat / CPR;
           const int c = flat - rl * CPR;
           const int srow = __shfl_sync(0xffffffffu, mine, rl);
-          const int r = 8 * pw + rl;
+          const int r = RW * pw + rl;
           const bool has = srow >= 0;
           const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * C::D + c * 8;
           cp_async_16(stage + (c >> 3) * C::ATOM + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
@@ -390,7 +399,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         cp_async_arrive_noinc(&kv_full[sl]);
       }
       cp_async_wait_all();
-    } else {
+    } else if (warp == C::MMA_WARP) {
       // ---------------------------------------------------------- MMA: S = Q K^T, M = 128
       if (lane == 0) {
         bool ok = mbar_wait(q_moved, 0, abort_flag);
@@ -429,7 +438,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     uint64_t* o_done = bars + 20;
     uint64_t* fin_ready = bars + 21;
     const uint32_t slot_free_peer = mapa_shared(smem_u32(smem + C::A_OFF_BAR + 12 * 8), partner);
-    if (warp == 13) {
+    if (warp == C::AUX_WARP) {
       // ---------------------------------------------------------- P copy: ring slot -> P stage
       // Runs up to NPS tiles ahead of the rescale warps and the MMA.
       bool ok = true;
@@ -476,15 +485,16 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&rescaled[ps]);  // also on failure: every wait stays bounded
       }
-    } else if (warp < 12) {
-      // ---------------------------------------------------------- gather the latent part (8 warps)
+    } else if (warp < C::MMA_WARP) {
+      // ---------------------------------------------------------- gather the latent part
       pdl_wait_prior();
       static_assert(C::DC / 8 == 64, "64 16-byte chunks per latent row");
+      constexpr int RW = C::ROWS_PER_GW;
       const int pw = warp - 4;
       const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * C::D;
       auto row_index = [&](int tile) -> int {
-        const int k = k_begin + tile * C::TK + 8 * pw + lane;
-        return (lane < 8 && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
+        const int k = k_begin + tile * C::TK + RW * pw + lane;
+        return (lane < RW && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
       };
       int nxt = row_index(0);
       for (int j = 0; j < n_tiles; ++j) {
@@ -494,13 +504,13 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         if (!mbar_wait_warp(&v_empty[sl], ((j / C::NVS) & 1) ^ 1u, abort_flag)) break;
         const int mine = (cur >= 0 && cur < len) ? cur : -1;  // the score CTA reports bad indices
         const uint32_t stage = smem_u32(smem + C::B_OFF_V + sl * C::V_BYTES);
-#pragma unroll 4
-        for (int q = 0; q < 16; ++q) {
+#pragma unroll 8
+        for (int q = 0; q < RW * 64 / 32; ++q) {
           const int flat = q * 32 + lane;
           const int rl = flat >> 6;
           const int c = flat & 63;
           const int srow = __shfl_sync(0xffffffffu, mine, rl);
-          const int r = 8 * pw + rl;
+          const int r = RW * pw + rl;
           const bool has = srow >= 0;
           const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * C::D + c * 8;
           cp_async_16(stage + (c >> 3) * C::ATOM + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
@@ -508,7 +518,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         cp_async_arrive_noinc(&v_full[sl]);
       }
       cp_async_wait_all();
-    } else {
+    } else if (warp == C::MMA_WARP) {
       // ---------------------------------------------------------- MMA: O += P V, M = 128
       if (lane == 0) {
         bool ok = true;
@@ -545,18 +555,27 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       __syncwarp();
     }
 
-    // ------------------------------------------------------------ epilogue (warps 0-11)
-    // O is final once the drain commit has landed. Warps w, w + 4 and w + 8
-    // read the same 32 TMEM lanes (32 (w % 4) ...) and split the 512 columns:
-    // 11, 11 and 10 chunks of 16.
-    if (warp < 12) {
-      const int h = (warp & 3) * 32 + lane;
-      const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-      const int third = warp >> 2;
-      const int c_lo = third * 176;
-      const int c_hi = third == 2 ? C::DC : c_lo + 176;
-      bool ok = mbar_wait_cluster_all(fin_ready, 0, abort_flag);
-      float2 ml = make_float2(-INFINITY, 0.0f);
+    // ------------------------------------------------------------ epilogue (warps 0-19)
+    // O is final once the drain commit has landed. Warps w, w + 4, ... read
+    // the same 32 TMEM lanes (32 (w % 4) ...) and split the 32 chunks of 16
+    // columns between them.
+    // With key splits, split s owns the head rows [128 s / S, 128 (s+1) / S):
+    // before the cluster barrier every value CTA writes the rows it does not
+    // own (unnormalised, with their (max, sum)) to the workspace; after it,
+    // each merges its own rows, read straight from tensor memory, with the
+    // other splits' copies of them and writes the output.
+    const int own_lo = split * C::M / S, own_hi = (split + 1) * C::M / S;
+    const int h = (warp & 3) * 32 + lane;
+    const bool owned = h >= own_lo && h < own_hi;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    constexpr int GROUPS = C::EPI_WARPS / 4;  // warps per TMEM sub-partition
+    const int third = warp >> 2;              // column group 0 .. GROUPS-1
+    const int c_lo = 16 * (third * (C::DC / 16) / GROUPS);
+    const int c_hi = 16 * ((third + 1) * (C::DC / 16) / GROUPS);
+    float2 ml = make_float2(-INFINITY, 0.0f);
+    bool ok = false;
+    if (warp < C::EPI_WARPS) {
+      ok = mbar_wait_cluster_all(fin_ready, 0, abort_flag);
       if (ok) ml = __ldcg(&fin[h]);
       if (ok) ok = mbar_wait_warp(drain, 0, abort_flag);
       if (ok) {
@@ -580,90 +599,107 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
             dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
           }
           if (third == 0 && p.lse) p.lse[row] = (ml.y > 0.0f) ? (ml.x + log2f(ml.y)) * 0.69314718055994531f : -INFINITY;
-        } else {
-          // this split's unnormalised rows ([column / 4][row] blocks) and statistics -> workspace
+        } else if (__any_sync(0xffffffffu, !owned)) {
+          // rows other splits own: unnormalised rows ([column / 4][row] blocks) and statistics -> workspace
           float4* po = reinterpret_cast<float4*>(p.part_o + pair * C::M * C::DC) + h;
 #pragma unroll 1
           for (int c = c_lo; c < c_hi; c += 16) {
             float o[16];
             tmem_ld16(tmem_base + lane_addr + c, o);
             tmem_wait_ld();
+            if (!owned) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              po[(c / 4 + u) * C::M] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+              for (int u = 0; u < 4; ++u)
+                po[(c / 4 + u) * C::M] = make_float4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+            }
           }
-          if (third == 0) p.part_ml[pair * C::M + h] = ml;
+          if (third == 0 && !owned) p.part_ml[pair * C::M + h] = ml;
         }
       }
     }
+    if (S > 1) {
+      cluster_sync_all();  // every split's rows for the others are in the workspace
+      if (warp < C::EPI_WARPS && ok && __any_sync(0xffffffffu, owned)) {
+        // merge the rows this split owns: its own (tensor memory) with the
+        // other splits' (workspace), with a running maximum
+        const int64_t grp = static_cast<int64_t>(t) * S;
+        float Mx = ml.x, L = ml.y;
+        if (!(L > 0.0f)) {
+          Mx = -INFINITY;
+          L = 0.0f;
+        }
+        float fo[C::MAX_SPLITS], fl = 1.0f;  // per-source factors onto the common maximum
+        {
+          float2 pm[C::MAX_SPLITS];
+          float nm = Mx;
+#pragma unroll
+          for (int sp = 0; sp < C::MAX_SPLITS; ++sp) {
+            pm[sp] = make_float2(-INFINITY, 0.0f);
+            if (sp < S && sp != split && owned) {
+              pm[sp] = __ldcg(&p.part_ml[(grp + sp) * C::M + h]);
+              if (!(pm[sp].y > 0.0f)) pm[sp] = make_float2(-INFINITY, 0.0f);
+              nm = fmaxf(nm, pm[sp].x);
+            }
+          }
+          const bool any = nm != -INFINITY;
+          fl = (any && L > 0.0f) ? exp2f(Mx - nm) : 0.0f;
+          float Lt = L * fl;
+#pragma unroll
+          for (int sp = 0; sp < C::MAX_SPLITS; ++sp) {
+            fo[sp] = (any && pm[sp].y > 0.0f) ? exp2f(pm[sp].x - nm) : 0.0f;
+            Lt += pm[sp].y * fo[sp];
+          }
+          Mx = nm;
+          L = Lt;
+        }
+        const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+        const int64_t row = static_cast<int64_t>(t) * C::M + h;
+#pragma unroll 1
+        for (int c = c_lo; c < c_hi; c += 16) {
+          float o[16];
+          tmem_ld16(tmem_base + lane_addr + c, o);
+          tmem_wait_ld();
+          if (owned) {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) o[u] *= fl;
+#pragma unroll
+            for (int sp = 0; sp < C::MAX_SPLITS; ++sp) {
+              if (sp < S && sp != split && fo[sp] != 0.0f) {
+                const float4* po = reinterpret_cast<const float4*>(p.part_o + (grp + sp) * C::M * C::DC) + h;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                  const float4 x = __ldcg(po + (c / 4 + u) * C::M);
+                  o[4 * u] = fmaf(x.x, fo[sp], o[4 * u]);
+                  o[4 * u + 1] = fmaf(x.y, fo[sp], o[4 * u + 1]);
+                  o[4 * u + 2] = fmaf(x.z, fo[sp], o[4 * u + 2]);
+                  o[4 * u + 3] = fmaf(x.w, fo[sp], o[4 * u + 3]);
+                }
+              }
+            }
+            uint32_t w8[8];
+#pragma unroll
+            for (int u = 0; u < 16; u += 2) {
+              const __nv_bfloat162 o2 = __floats2bfloat162_rn(o[u] * inv, o[u + 1] * inv);
+              w8[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(p.out + row * C::DC + c);
+            dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+            dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+          }
+        }
+        if (third == 0 && owned && p.lse) p.lse[row] = (L > 0.0f) ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
   }
+  if (score_cta && S > 1) cluster_sync_all();  // pairs with the value CTAs' barrier above
 
   // The next kernel of the stream may be scheduled now (see the indexer).
   pdl_launch_dependents();
 
-  if (S > 1) {
-    // ---------------- merge the key-split partials of the value CTAs
-    cluster_sync_all();
-    if (!score_cta) {
-      const int64_t grp = static_cast<int64_t>(t) * S;
-      constexpr int SL = 16, NSL = C::DC / SL;
-      const int owned = (C::M - split + S - 1) / S;  // heads split, split + S, ...
-      for (int item = threadIdx.x; item < owned * NSL; item += C::THREADS) {
-        const int hl = split + S * (item % owned);
-        const int c0 = (item / owned) * SL;
-        float Mx = -INFINITY, L = 0.0f, acc[SL];
-#pragma unroll
-        for (int u = 0; u < SL; ++u) acc[u] = 0.0f;
-        for (int sb = 0; sb < S; sb += 2) {
-          float2 ml[2];
-          float4 x[2][SL / 4];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            if (sb + u < S) {
-              ml[u] = __ldcg(&p.part_ml[(grp + sb + u) * C::M + hl]);
-              const float4* po = reinterpret_cast<const float4*>(p.part_o + (grp + sb + u) * C::M * C::DC) + hl;
-#pragma unroll
-              for (int v4 = 0; v4 < SL / 4; ++v4) x[u][v4] = __ldcg(po + (c0 / 4 + v4) * C::M);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            if (sb + u < S && ml[u].y > 0.0f) {
-              const float nm = fmaxf(Mx, ml[u].x);
-              const float fo = exp2f(Mx - nm);
-              const float fn = exp2f(ml[u].x - nm);
-              L = L * fo + ml[u].y * fn;
-#pragma unroll
-              for (int v4 = 0; v4 < SL / 4; ++v4) {
-                acc[4 * v4 + 0] = acc[4 * v4 + 0] * fo + x[u][v4].x * fn;
-                acc[4 * v4 + 1] = acc[4 * v4 + 1] * fo + x[u][v4].y * fn;
-                acc[4 * v4 + 2] = acc[4 * v4 + 2] * fo + x[u][v4].z * fn;
-                acc[4 * v4 + 3] = acc[4 * v4 + 3] * fo + x[u][v4].w * fn;
-              }
-              Mx = nm;
-            }
-          }
-        }
-        const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-        const int64_t row = static_cast<int64_t>(t) * C::M + hl;
-        uint32_t w[SL / 2];
-#pragma unroll
-        for (int u = 0; u < SL; u += 2) {
-          const __nv_bfloat162 o2 = __floats2bfloat162_rn(acc[u] * inv, acc[u + 1] * inv);
-          w[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(p.out + row * C::DC + c0);
-#pragma unroll
-        for (int u = 0; u < SL / 8; ++u) dst[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        if (c0 == 0 && p.lse) p.lse[row] = (L > 0.0f) ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
-      }
-    }
-  }
-
   // No CTA may retire while its partner can still address its shared memory.
   tc_fence_before();
   cluster_sync_all();
-  if (warp == 12) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }

@@ -160,3 +160,43 @@ def test_attention_workspace_layout(lib):
     b1 = _batch(num_q=1, batch=1, max_seq_len=8192)
     one = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b1), 2048, 64, 128)
     assert one == ring_fin + 4 * 128 * (512 * 4 + 8)
+
+
+def _header_shapes():
+    """The supported-shape block of include/dsa.h, parsed."""
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    pairs = lambda line: {tuple(int(v) for v in m) for m in re.findall(r"\((\d+),\s*(\d+)\)", line)}
+    idx_line = re.search(r"indexer \(H_I, d_I\):(.*)", text).group(1)
+    mla_line = re.search(r"MLA \(d_latent, d_rope\):(.*)", text).group(1)
+    heads_line = re.search(r"MLA heads H:(.*)", text).group(1)
+    k_line = re.search(r"top-K k:(.*)", text).group(1)
+    heads = set()
+    for lo, hi in re.findall(r"(\d+)\.\.(\d+)", heads_line):
+        heads |= set(range(int(lo), int(hi) + 1))
+    heads |= {int(v) for v in re.findall(r"or (\d+)", heads_line)}
+    k_lo, k_hi = (int(v) for v in re.search(r"(\d+)\.\.(\d+)", k_line).groups())
+    return pairs(idx_line), pairs(mla_line), heads, (k_lo, k_hi)
+
+
+def test_header_supported_shapes_match_validation(lib):
+    """Every shape the header lists passes validation (an empty batch then
+    returns DSA_OK with nothing enqueued) and every shape it does not list is
+    rejected with DSA_ERR_UNSUPPORTED_SHAPE."""
+    idx_pairs, mla_pairs, heads, (k_lo, k_hi) = _header_shapes()
+    assert idx_pairs == {(4, 32), (4, 128), (64, 32), (64, 128)}
+    empty = _batch(num_q=0)
+    for hi in (1, 2, 4, 8, 16, 32, 48, 64, 96, 128):
+        for di in (16, 32, 64, 96, 128, 256):
+            want = B.DSA_OK if (hi, di) in idx_pairs else B.DSA_ERR_UNSUPPORTED_SHAPE
+            assert _scores(lib, empty, _idx_in(n_heads=hi, head_dim=di, scale_group=di)) == want, (hi, di)
+    for dl, dr in [(512, 64), (64, 16), (512, 0), (256, 64), (64, 64), (128, 16), (576, 0)]:
+        for h in (1, 4, 32, 63, 64, 65, 96, 127, 128, 129, 192, 256):
+            want = B.DSA_OK if ((dl, dr) in mla_pairs and h in heads) else B.DSA_ERR_UNSUPPORTED_SHAPE
+            got = lib.dsa_sparse_mla_attn(ctypes.byref(empty), ctypes.byref(_mla_in(n_heads=h, d_latent=dl, d_rope=dr)),
+                                          FAKE, 64, FAKE, None, None, 0, None)
+            assert got == want, (dl, dr, h)
+    for k in (k_lo - 1, k_lo, 2, 1024, k_hi, k_hi + 1):
+        want = B.DSA_OK if k_lo <= k <= k_hi else B.DSA_ERR_UNSUPPORTED_SHAPE
+        assert lib.dsa_topk(ctypes.byref(empty), FAKE, 256, k, FAKE, None, 0, None) == want, k
+        got = lib.dsa_sparse_mla_attn(ctypes.byref(empty), ctypes.byref(_mla_in()), FAKE, k, FAKE, None, None, 0, None)
+        assert got == want, k

@@ -221,6 +221,17 @@ def test_topk_long_rows_and_crowded_threshold_bin():
     assert list(idx[2]) == list(range(2048))
 
 
+def test_topk_rows_beyond_the_bitmap_budget():
+    """Rows so long (800 000 positions) that two position bitmaps no longer fit
+    in shared memory: the one-pass-per-digit radix kernel streams the row from
+    memory for each 8-bit digit."""
+    rng = np.random.default_rng(17)
+    rows = [W.bf16_round(rng.standard_normal(800_000).astype(np.float32) * 8),
+            np.float32(rng.integers(-40, 40, 790_001))]
+    idx, sc, lens = _topk_rows(rows, 2048)
+    assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
+
+
 # ----------------------------------------------------------------------------- sparse MLA
 
 def _mla_check(wl, idx_np):
