@@ -204,7 +204,8 @@ MlaPlan pipe_plan_with(int T, int K, MaxClusters max_clusters) {
   const int tiles = (K + C::TK - 1) / C::TK;
   int best = 1;
   int64_t best_cost = -1;
-  for (int sp = 1; sp <= C::MAX_SPLITS && sp <= tiles; ++sp) {
+  for (int sp = 1; sp <= C::MAX_SPLITS && sp <= tiles; sp *= 2) {  // 1, 2, 4: a split owns 128 / S rows
+    if ((sp - 1) * ((tiles + sp - 1) / sp) >= tiles) continue;     // the last split would get no tile
     const int mc = max_clusters(sp);
     if (mc < 1) break;
     const int64_t waves = (static_cast<int64_t>(T) + mc - 1) / mc;
@@ -215,8 +216,7 @@ MlaPlan pipe_plan_with(int T, int K, MaxClusters max_clusters) {
     }
   }
   const int tps = (tiles + best - 1) / best;
-  const int splits = (tiles + tps - 1) / tps;
-  return MlaPlan{splits, tps * C::TK};
+  return MlaPlan{best, tps * C::TK};  // the last split may get fewer tiles (never none: best <= tiles)
 }
 
 MlaPlan pipe_plan(int T, int K, int sms) {
@@ -506,8 +506,10 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
   if (!ws || ws_bytes < need)
     return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "attention workspace %zu < %zu bytes", ws_bytes, need);
   if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
-  CUtensorMap qmap;
+  CUtensorMap qmap, kvmap;
   if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(T) * C::M, C::D, C::M)) != DSA_OK) return s;
+  if ((s = make_bf16_rows_map(&kvmap, in->kv, static_cast<int64_t>(bt->batch) * bt->max_seq_len, C::D, 1)) != DSA_OK)
+    return s;
   PipeParams p;
   p.cu_q = bt->cu_q;
   p.seq_lens = bt->seq_lens;
@@ -533,6 +535,23 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
     p.part_o = reinterpret_cast<float*>(w);
     p.part_ml = reinterpret_cast<float2*>(w + align256(rows * C::DC * sizeof(float)));
   }
+  // the split partials as a 2-D fp32 tensor: x = head row x 4 (512 floats, a
+  // [row][4] block per 4 output columns), y = (pair, column / 4)
+  CUtensorMap pmap;
+  std::memset(&pmap, 0, sizeof(pmap));
+  if (pl.splits > 1) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C::M) * 4,
+                                static_cast<cuuint64_t>(T) * pl.splits * (C::DC / 4)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C::M) * 4 * sizeof(float)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::M / pl.splits * 4), static_cast<cuuint32_t>(C::DC / 4)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(&pmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.part_o, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled (partials) failed (%d)", static_cast<int>(r));
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pl.splits, T, 1);
   cfg.blockDim = dim3(C::THREADS);
@@ -553,7 +572,7 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
   cfg.attrs = attr;
   cfg.numAttrs = na;
   const cudaError_t e =
-      cudaLaunchKernelEx(&cfg, sparse_mla_pipe_kernel, static_cast<const __nv_bfloat16*>(in->kv), qmap, p);
+      cudaLaunchKernelEx(&cfg, sparse_mla_pipe_kernel, kvmap, qmap, pmap, p);
   if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla_pipe launch: %s", cudaGetErrorString(e));
   return check_launch("sparse_mla_pipe");
 }

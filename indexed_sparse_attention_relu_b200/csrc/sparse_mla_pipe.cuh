@@ -77,7 +77,12 @@ struct PipeCfg {
   static constexpr int EPI_WARPS = 4 + NGATHER;
   static constexpr int NUM_WARPS = AUX_WARP + 1;
   static constexpr int THREADS = NUM_WARPS * 32;
-  static constexpr int MAX_SPLITS = 4;
+  static constexpr int MAX_SPLITS = 4;                  // 1, 2 or 4 (a split owns 128 / S head rows)
+  // Merge: the other splits' copies of a split's rows arrive by TMA into the
+  // value CTA's (then idle) V stages, one box of 128 / S rows x 512 columns
+  // per other split (stored [column / 4][row][4] like the workspace).
+  static constexpr int MERGE_BAR = 19;
+  static constexpr int box_bytes(int S) { return (M / S) * DC * 4; }
   // score CTA shared memory
   static constexpr int A_OFF_K = 0;
   static constexpr int A_OFF_BAR = NKS * K_BYTES;
@@ -86,14 +91,25 @@ struct PipeCfg {
   static constexpr int B_OFF_V = NPS * P_STAGE;
   static constexpr int B_OFF_BAR = B_OFF_V + NVS * V_BYTES;
   static constexpr int NUM_BARS = 24;
-  static constexpr int SMEM_BYTES = (A_OFF_BAR > B_OFF_BAR ? A_OFF_BAR : B_OFF_BAR) + NUM_BARS * 8 + 16;
+  static constexpr int MISC_BYTES = 32;
+  // score CTA: the split's selected indices, staged once (a load issued while
+  // the gathers stream queues behind them for microseconds)
+  static constexpr int A_OFF_IDX = A_OFF_BAR + NUM_BARS * 8 + MISC_BYTES;
+  static constexpr int MAX_K = 2048;
+  static constexpr int A_END = A_OFF_IDX + MAX_K * 4;
+  static constexpr int B_END = B_OFF_BAR + NUM_BARS * 8 + MISC_BYTES;
+  static constexpr int SMEM_BYTES = A_END > B_END ? A_END : B_END;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(M, TK, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(M, 256, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(COL_Q + D / 2 <= 512, "TMEM budget of the score CTA");
   static_assert(2 * K_BYTES >= 9 * Q_ATOM, "Q is staged in gather stages 1 and 2");
   static_assert(P_IMG % 1024 == 0 && SLOT_BYTES % 16 == 0, "ring slot layout");
+  static_assert(B_OFF_V % 1024 == 0, "TMA destination alignment");
 };
+static_assert(PipeCfg::box_bytes(2) <= PipeCfg::NVS * PipeCfg::V_BYTES &&
+                  (PipeCfg::MAX_SPLITS - 1) * PipeCfg::box_bytes(PipeCfg::MAX_SPLITS) <= PipeCfg::NVS * PipeCfg::V_BYTES,
+              "merge boxes fit in the V stages");
 
 __device__ __forceinline__ void tmem_st16w(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
@@ -110,8 +126,8 @@ __device__ __forceinline__ bool mbar_wait_cluster_all(uint64_t* bar, uint32_t pa
 }
 
 __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
-    sparse_mla_pipe_kernel(const __nv_bfloat16* __restrict__ kv, const __grid_constant__ CUtensorMap qmap,
-                           const PipeParams p) {
+    sparse_mla_pipe_kernel(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap,
+                           const __grid_constant__ CUtensorMap pmap, const PipeParams p) {
   using C = PipeCfg;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {  // same in every CTA: all leave or none
@@ -141,12 +157,14 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
   // value CTA: [0,3) v_full, [3,6) v_empty, [6,8) p_full, [8,10) p_empty, [12,16) p_ready (remote
   //            arrivals from the score CTA), 16 drain, [17,19) rescaled (per P stage), 20 o_done,
   //            21 fin_ready (remote)
-  int32_t* misc = reinterpret_cast<int32_t*>(bars + C::NUM_BARS);  // [0] TMEM base, [1] abort, [2] SM id
+  // [0] TMEM base, [1] abort, [2] SM id, [4..6) per-tile go flags of the gather warps
+  int32_t* misc = reinterpret_cast<int32_t*>(bars + C::NUM_BARS);
+  int32_t* sidx = reinterpret_cast<int32_t*>(smem + C::A_OFF_IDX);  // score CTA only
   volatile int* abort_flag = misc + 1;
   if (threadIdx.x == 0) {
     if (score_cta) {
       for (int i = 0; i < C::NKS; ++i) {
-        mbar_init(&bars[i], C::NGATHER * 32);  // one asynchronous arrival per gather thread
+        mbar_init(&bars[i], 1);  // the gather leader's arrival (+ the row gathers' bytes)
         mbar_init(&bars[3 + i], 1);
       }
       mbar_init(&bars[6], 1);
@@ -163,7 +181,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       mbar_init(&bars[21], 128);
     } else {
       for (int i = 0; i < C::NVS; ++i) {
-        mbar_init(&bars[i], C::NGATHER * 32);
+        mbar_init(&bars[i], 1);
         mbar_init(&bars[3 + i], 1);
       }
       for (int i = 0; i < C::NPS; ++i) {
@@ -176,6 +194,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       mbar_init(&bars[18], 4);
       mbar_init(&bars[20], 1);
       mbar_init(&bars[21], 1);
+      mbar_init(&bars[C::MERGE_BAR], 1);
     }
     misc[1] = 0;
     uint32_t smid;
@@ -183,6 +202,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     misc[2] = static_cast<int32_t>(smid);
     fence_mbar_init();
     if (score_cta) prefetch_tensormap(&qmap);
+    prefetch_tensormap(&kvmap);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(reinterpret_cast<uint32_t*>(misc), 512);
@@ -253,17 +273,13 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_moved);  // also on failure: every wait stays bounded
-      pdl_wait_prior();  // the selected indices (Top-K output) are complete from here on
+      named_bar_sync(2, 32 * (4 + C::NGATHER));  // the gather warps have staged the indices
 
       float m = -INFINITY, l = 0.0f;
-      auto idx_at = [&](int k) -> int { return k < k_end ? ld_dep(idx_row + k) : -1; };
-      int i0n = idx_at(k_begin + lane), i1n = idx_at(k_begin + 32 + lane);
+      const int nk = k_end - k_begin;
       for (int j = 0; j < n_tiles; ++j) {
-        const int i0 = i0n, i1 = i1n;
-        if (j + 1 < n_tiles) {
-          i0n = idx_at(k_begin + (j + 1) * C::TK + lane);
-          i1n = idx_at(k_begin + (j + 1) * C::TK + 32 + lane);
-        }
+        const int i0 = (j * C::TK + lane < nk) ? sidx[j * C::TK + lane] : -1;
+        const int i1 = (j * C::TK + 32 + lane < nk) ? sidx[j * C::TK + 32 + lane] : -1;
         const unsigned v0 = __ballot_sync(0xffffffffu, i0 >= 0 && i0 < len);
         const unsigned v1 = __ballot_sync(0xffffffffu, i1 >= 0 && i1 < len);
         float v[64];
@@ -363,42 +379,78 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       __syncwarp();
     } else if (warp < C::MMA_WARP) {
       // ---------------------------------------------------------- gather whole rows
-      pdl_wait_prior();
-      constexpr int CPR = C::D / 8;  // 72 chunks per row
-      constexpr int RW = C::ROWS_PER_GW;
-      const int pw = warp - 4;
-      const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * C::D;
-      auto row_index = [&](int tile) -> int {
-        const int k = k_begin + tile * C::TK + RW * pw + lane;
-        return (lane < RW && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
-      };
-      int nxt = row_index(0);
-      bool ok = true;
-      for (int j = 0; j < n_tiles && ok; ++j) {
-        const int sl = j % C::NKS;
-        const int cur = nxt;
-        nxt = row_index(j + 1);
-        if (j == 1) ok = mbar_wait_warp(q_moved, 0, abort_flag);  // stages 1, 2 hold Q until then
-        if (ok) ok = mbar_wait_warp(&kv_empty[sl], ((j / C::NKS) & 1) ^ 1u, abort_flag);
-        if (!ok) break;
-        const bool okr = cur >= 0 && cur < len;
-        if (lane < RW && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
-        const int mine = okr ? cur : -1;
-        const uint32_t stage = smem_u32(smem + C::A_OFF_K + sl * C::K_BYTES);
-#pragma unroll 9
-        for (int q = 0; q < RW * CPR / 32; ++q) {
-          const int flat = q * 32 + lane;
-          const int rl = flat / CPR;
-          const int c = flat - rl * CPR;
-          const int srow = __shfl_sync(0xffffffffu, mine, rl);
-          const int r = RW * pw + rl;
-          const bool has = srow >= 0;
-          const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * C::D + c * 8;
-          cp_async_16(stage + (c >> 3) * C::ATOM + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
+      // TMA row gathers (tile::gather4: four rows x one 64-dim atom column per
+      // op, placed in the 128-byte-swizzled K-major layout by the copy engine):
+      // 16 row groups x 9 atom columns = 144 ops per tile, one per gather
+      // thread. A leader waits for the stage and arms its barrier; the others
+      // learn through a per-tile flag whether to go on, so every tile is
+      // issued whole or not at all. Invalid rows (-1, or outside the
+      // sequence) fetch the sequence's row 0 instead: their logits are masked
+      // to -inf below and their P is 0.
+      pdl_wait_prior();  // the selected indices (Top-K output) are complete from here on
+      const int gl = threadIdx.x - 4 * 32;  // 0 .. 32 * NGATHER - 1
+      const bool leader = gl == 0;
+      const bool active = gl < 16 * 9;
+      const int g = gl / 9, a = gl - (gl / 9) * 9;
+      const int32_t row0 = b * p.L_max;
+      {
+        // stage this split's indices (eight independent loads in flight per thread)
+        const int nk = k_end - k_begin;
+        constexpr int GT = 32 * C::NGATHER;
+        for (int base = 0; base < nk; base += 8 * GT) {
+          int v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = base + u * GT + gl;
+            v[u] = i < nk ? ld_dep(idx_row + k_begin + i) : -1;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int i = base + u * GT + gl;
+            if (i < nk) sidx[i] = v[u];
+          }
         }
-        cp_async_arrive_noinc(&kv_full[sl]);
       }
-      cp_async_wait_all();
+      named_bar_sync(2, 32 * (4 + C::NGATHER));  // with the softmax warps
+      const int nk = k_end - k_begin;
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int sl = j % C::NKS;
+        int cur[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int kk = j * C::TK + 4 * g + i;
+          cur[i] = (active && kk < nk) ? sidx[kk] : -1;
+        }
+        if (leader) {
+          bool ok = true;
+          if (j == 1) ok = mbar_wait(q_moved, 0, abort_flag);  // stages 1, 2 hold Q until then
+          if (ok) ok = mbar_wait(&kv_empty[sl], ((j / C::NKS) & 1) ^ 1u, abort_flag);
+          if (ok) mbar_arrive_expect_tx(&kv_full[sl], C::K_BYTES);
+          reinterpret_cast<volatile int*>(misc)[4 + (j & 1)] = ok ? 1 : 0;
+        }
+        named_bar_sync(1, 32 * C::NGATHER);
+        if (!reinterpret_cast<volatile int*>(misc)[4 + (j & 1)]) break;
+        if (active) {
+          int y[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const bool v = cur[i] >= 0 && cur[i] < len;
+            if (a == 0 && cur[i] != -1 && !v) set_device_status(DSA_ERR_DEVICE_INDEX);
+            y[i] = row0 + (v ? cur[i] : 0);
+          }
+          tma_gather4(smem_u32(smem + C::A_OFF_K + sl * C::K_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0], y[1],
+                      y[2], y[3], &kv_full[sl]);
+        }
+        ++issued;
+      }
+      // every tile issued must land before the CTA can retire
+      if (leader) {
+        for (int j = issued > C::NKS ? issued - C::NKS : 0; j < issued; ++j) {
+          volatile int never = 0;
+          mbar_wait(&kv_full[j % C::NKS], (j / C::NKS) & 1, &never);
+        }
+      }
     } else if (warp == C::MMA_WARP) {
       // ---------------------------------------------------------- MMA: S = Q K^T, M = 128
       if (lane == 0) {
@@ -487,37 +539,64 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       }
     } else if (warp < C::MMA_WARP) {
       // ---------------------------------------------------------- gather the latent part
+      // The same TMA row gathers for atom columns 0-7 (the 512 latent dims):
+      // 16 row groups x 8 = 128 ops per tile (the score CTA reports bad indices).
+      // Indices are read four tiles ahead (a load issued while the gathers
+      // stream queues behind them for microseconds).
       pdl_wait_prior();
-      static_assert(C::DC / 8 == 64, "64 16-byte chunks per latent row");
-      constexpr int RW = C::ROWS_PER_GW;
-      const int pw = warp - 4;
-      const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * C::D;
-      auto row_index = [&](int tile) -> int {
-        const int k = k_begin + tile * C::TK + RW * pw + lane;
-        return (lane < RW && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
-      };
-      int nxt = row_index(0);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int sl = j % C::NVS;
-        const int cur = nxt;
-        nxt = row_index(j + 1);
-        if (!mbar_wait_warp(&v_empty[sl], ((j / C::NVS) & 1) ^ 1u, abort_flag)) break;
-        const int mine = (cur >= 0 && cur < len) ? cur : -1;  // the score CTA reports bad indices
-        const uint32_t stage = smem_u32(smem + C::B_OFF_V + sl * C::V_BYTES);
-#pragma unroll 8
-        for (int q = 0; q < RW * 64 / 32; ++q) {
-          const int flat = q * 32 + lane;
-          const int rl = flat >> 6;
-          const int c = flat & 63;
-          const int srow = __shfl_sync(0xffffffffu, mine, rl);
-          const int r = RW * pw + rl;
-          const bool has = srow >= 0;
-          const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * C::D + c * 8;
-          cp_async_16(stage + (c >> 3) * C::ATOM + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
+      const int gl = threadIdx.x - 4 * 32;
+      const bool leader = gl == 0;
+      const bool active = gl < 16 * 8;
+      const int g = gl >> 3, a = gl & 7;
+      const int32_t row0 = b * p.L_max;
+      auto load_rows = [&](int tile, int (&y)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int k = k_begin + tile * C::TK + 4 * g + i;
+          y[i] = (active && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
         }
-        cp_async_arrive_noinc(&v_full[sl]);
+      };
+      int r0[4], r1[4], r2[4], r3[4];
+      load_rows(0, r0);
+      load_rows(1, r1);
+      load_rows(2, r2);
+      load_rows(3, r3);
+      int issued = 0;
+      bool stop = false;
+      for (int j0 = 0; j0 < n_tiles && !stop; j0 += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = j0 + u;
+          if (j >= n_tiles || stop) break;
+          int (&cur)[4] = u == 0 ? r0 : u == 1 ? r1 : u == 2 ? r2 : r3;
+          const int sl = j % C::NVS;
+          if (leader) {
+            const bool ok = mbar_wait(&v_empty[sl], ((j / C::NVS) & 1) ^ 1u, abort_flag);
+            if (ok) mbar_arrive_expect_tx(&v_full[sl], C::V_BYTES);
+            reinterpret_cast<volatile int*>(misc)[4 + (j & 1)] = ok ? 1 : 0;
+          }
+          named_bar_sync(1, 32 * C::NGATHER);
+          if (!reinterpret_cast<volatile int*>(misc)[4 + (j & 1)]) {
+            stop = true;
+            break;
+          }
+          if (active) {
+            int y[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[i] = row0 + ((cur[i] >= 0 && cur[i] < len) ? cur[i] : 0);
+            tma_gather4(smem_u32(smem + C::B_OFF_V + sl * C::V_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0],
+                        y[1], y[2], y[3], &v_full[sl]);
+          }
+          ++issued;
+          load_rows(j + 4, cur);
+        }
       }
-      cp_async_wait_all();
+      if (leader) {
+        for (int j = issued > C::NVS ? issued - C::NVS : 0; j < issued; ++j) {
+          volatile int never = 0;
+          mbar_wait(&v_full[j % C::NVS], (j / C::NVS) & 1, &never);
+        }
+      }
     } else if (warp == C::MMA_WARP) {
       // ---------------------------------------------------------- MMA: O += P V, M = 128
       if (lane == 0) {
@@ -591,7 +670,9 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
             uint32_t w8[8];
 #pragma unroll
             for (int u = 0; u < 16; u += 2) {
-              const __nv_bfloat162 o2 = __floats2bfloat162_rn(o[u] * inv, o[u + 1] * inv);
+              // a row with no valid key writes zeros whatever its O holds
+              const __nv_bfloat162 o2 = inv != 0.0f ? __floats2bfloat162_rn(o[u] * inv, o[u + 1] * inv)
+                                                    : __floats2bfloat162_rn(0.0f, 0.0f);
               w8[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
             }
             uint4* dst = reinterpret_cast<uint4*>(p.out + row * C::DC + c);
@@ -614,15 +695,29 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
             }
           }
           if (third == 0 && !owned) p.part_ml[pair * C::M + h] = ml;
+          fence_proxy_async_global();  // the owner reads these rows through the async proxy (TMA)
         }
       }
     }
     if (S > 1) {
       cluster_sync_all();  // every split's rows for the others are in the workspace
+      uint64_t* merge_full = bars + C::MERGE_BAR;
+      const int own_n = C::M / S;
+      const int64_t grp = static_cast<int64_t>(t) * S;
+      const int issuer_warp = own_lo / 32;  // the first warp of the owned rows
+      if (warp == issuer_warp && lane == 0 && ok) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(merge_full, (S - 1) * C::box_bytes(S));
+        for (int sp = 0, i = 0; sp < S; ++sp) {
+          if (sp == split) continue;
+          tma_load_2d(smem_u32(smem + C::B_OFF_V + i * C::box_bytes(S)), &pmap, own_lo * 4,
+                      static_cast<int32_t>((grp + sp) * (C::DC / 4)), merge_full);
+          ++i;
+        }
+      }
       if (warp < C::EPI_WARPS && ok && __any_sync(0xffffffffu, owned)) {
         // merge the rows this split owns: its own (tensor memory) with the
-        // other splits' (workspace), with a running maximum
-        const int64_t grp = static_cast<int64_t>(t) * S;
+        // other splits' (shared memory), with a running maximum
         float Mx = ml.x, L = ml.y;
         if (!(L > 0.0f)) {
           Mx = -INFINITY;
@@ -654,41 +749,52 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         }
         const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
         const int64_t row = static_cast<int64_t>(t) * C::M + h;
+        const int hr = owned ? h - own_lo : 0;
+        if (mbar_wait_warp(merge_full, 0, abort_flag)) {
 #pragma unroll 1
-        for (int c = c_lo; c < c_hi; c += 16) {
-          float o[16];
-          tmem_ld16(tmem_base + lane_addr + c, o);
-          tmem_wait_ld();
-          if (owned) {
+          for (int c = c_lo; c < c_hi; c += 16) {
+            float o[16];
+            tmem_ld16(tmem_base + lane_addr + c, o);
+            tmem_wait_ld();
+            if (owned) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u) o[u] *= fl;
+              for (int u = 0; u < 16; ++u) o[u] *= fl;
 #pragma unroll
-            for (int sp = 0; sp < C::MAX_SPLITS; ++sp) {
-              if (sp < S && sp != split && fo[sp] != 0.0f) {
-                const float4* po = reinterpret_cast<const float4*>(p.part_o + (grp + sp) * C::M * C::DC) + h;
+              for (int sp = 0, i = 0; sp < C::MAX_SPLITS; ++sp) {
+                if (sp >= S || sp == split) continue;
+                const float4* px = reinterpret_cast<const float4*>(smem + C::B_OFF_V + i * C::box_bytes(S)) + hr;
+                ++i;
+                if (fo[sp] == 0.0f) continue;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                  const float4 x = __ldcg(po + (c / 4 + u) * C::M);
+                  const float4 x = px[(c / 4 + u) * own_n];
                   o[4 * u] = fmaf(x.x, fo[sp], o[4 * u]);
                   o[4 * u + 1] = fmaf(x.y, fo[sp], o[4 * u + 1]);
                   o[4 * u + 2] = fmaf(x.z, fo[sp], o[4 * u + 2]);
                   o[4 * u + 3] = fmaf(x.w, fo[sp], o[4 * u + 3]);
                 }
               }
-            }
-            uint32_t w8[8];
+              uint32_t w8[8];
 #pragma unroll
-            for (int u = 0; u < 16; u += 2) {
-              const __nv_bfloat162 o2 = __floats2bfloat162_rn(o[u] * inv, o[u + 1] * inv);
-              w8[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
+              for (int u = 0; u < 16; u += 2) {
+                // a row with no valid key writes zeros whatever its O holds
+                const __nv_bfloat162 o2 = inv != 0.0f ? __floats2bfloat162_rn(o[u] * inv, o[u + 1] * inv)
+                                                      : __floats2bfloat162_rn(0.0f, 0.0f);
+                w8[u / 2] = *reinterpret_cast<const uint32_t*>(&o2);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(p.out + row * C::DC + c);
+              dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+              dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
             }
-            uint4* dst = reinterpret_cast<uint4*>(p.out + row * C::DC + c);
-            dst[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
-            dst[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
           }
+          if (third == 0 && owned && p.lse) p.lse[row] = (L > 0.0f) ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
         }
-        if (third == 0 && owned && p.lse) p.lse[row] = (L > 0.0f) ? (Mx + log2f(L)) * 0.69314718055994531f : -INFINITY;
       }
+      if (warp == issuer_warp && lane == 0 && ok) {
+        volatile int never = 0;  // the copies must land before the CTA can retire
+        mbar_wait(merge_full, 0, &never);
+      }
+      __syncwarp();
     }
   }
   if (score_cta && S > 1) cluster_sync_all();  // pairs with the value CTAs' barrier above
