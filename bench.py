@@ -5,8 +5,12 @@ Default workload: decode, batch 32 x 8192 context, one new token each
 (H_I=64, d_I=128, K=2048, 128 MLA heads, 512+64 latent dims, BF16), timed as
 one ``dsa_fused_decode`` call per step through the C ABI. Prints one JSON line.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c3|c4|c5]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c3|c4|c5] [--extra c3,c4,c5]
   python bench.py --impl reference ...     # the CPU oracle, timed on host cores
+
+The JSON line's headline is the decode workload; ``configs`` adds one block
+per extra workload (the ragged FP8-key decode against the HBM roofline, the
+prefills against the dense tensor-core peak), each graph-timed the same way.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronize, timed with CUDA events on the launch stream; max over
@@ -54,6 +58,27 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def _peak_tflops():
+    """(burst, sustained) dense bf16 TFLOP/s measured on this machine, or the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
+def algorithmic_flops(wl, n_selected: int):
+    """Tensor-core FLOPs each stage must do (2 per multiply-add): the indexer's
+    q_I . k_I products over every causal candidate and head, and the attention's
+    QK^T (D dims) and PV (d_c dims) over every selected row and head."""
+    nv = wl.n_valid().astype(np.int64)
+    idx = int(nv.sum()) * wl.HI * wl.dI * 2
+    attn = int(n_selected) * wl.H * (wl.D + wl.dc) * 2
+    return {"indexer": idx, "sparse_mla": attn, "step": idx + attn}
+
+
 def algorithmic_bytes(wl, n_selected: int):
     """Bytes each stage must move at least once (inputs read + outputs written).
 
@@ -76,21 +101,24 @@ def algorithmic_bytes(wl, n_selected: int):
 class ClockSampler:
     """SM clock, power and clock-event reasons sampled during the timed region.
 
-    Reads (never sets) NVML in a background thread every 2 ms, so even a
-    few-millisecond timed region gets samples; falls back to polling
-    nvidia-smi when NVML is unavailable."""
+    Reads (never sets) NVML in a background thread every 0.2 ms from before the
+    timed region until after it; mark() brackets the region with host
+    timestamps and summary() keeps only the samples taken inside it."""
 
     # NVML clock-event reason bits
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, torch_device):
+    def __init__(self, torch_device, period_s: float = 0.0002):
         self.dev = torch_device
         self.samples = []
         self.stop = False
         self.thread = None
         self.handle = None
         self.error = None
+        self.period = period_s
+        self.t0 = self.t1 = None
+        self.max_mhz = None
 
     def __enter__(self):
         import threading
@@ -104,35 +132,47 @@ class ClockSampler:
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
             get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
                 pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            started = threading.Event()
 
             def loop():
                 while not self.stop:
                     try:
-                        self.samples.append((pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM),
+                        self.samples.append((time.perf_counter(),
+                                             pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM),
                                              pynvml.nvmlDeviceGetPowerUsage(self.handle) / 1000.0,
                                              int(get_reasons(self.handle))))
                     except Exception as e:  # keep sampling; record the first problem
                         self.error = self.error or repr(e)
-                    time.sleep(0.002)
+                    started.set()
+                    time.sleep(self.period)
 
             self.thread = threading.Thread(target=loop, daemon=True)
             self.thread.start()
+            started.wait(timeout=2.0)   # the sampler is running before the region starts
         except Exception as e:
             self.error = repr(e)
         return self
 
+    def mark(self, which: str):
+        if which == "start":
+            self.t0 = time.perf_counter()
+        else:
+            self.t1 = time.perf_counter()
+
     def __exit__(self, *a):
+        time.sleep(2 * self.period)
         self.stop = True
         if self.thread is not None:
             self.thread.join(timeout=5)
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": self.error}
-        seen = sorted({name for _, _, r in self.samples for bit, name in self.REASONS.items() if r & bit})
-        return {"sm_mhz": statistics.median(c for c, _, _ in self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": seen, "samples": len(self.samples),
-                "power_w_max": max(p for _, p, _ in self.samples)}
+        inside = [s for s in self.samples
+                  if self.t0 is None or self.t1 is None or self.t0 <= s[0] <= self.t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "note": self.error}
+        seen = sorted({name for _, _, _, r in inside for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(c for _, c, _, _ in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": seen, "samples": len(inside), "power_w_max": max(p for _, _, p, _ in inside)}
 
 
 def run_cpu_oracle(wl, n_tokens: int, seed: int = 0, min_seconds: float = 0.0):
@@ -185,6 +225,203 @@ def reference_arm(args, rank: int):
     print(json.dumps(line), flush=True)
 
 
+def _stage_events(B, steps):
+    import torch
+    return [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+
+
+class Runner:
+    """One workload resident on the device in rotating copies, run through
+    dsa_fused_decode (the whole chain as one C-ABI call per step)."""
+
+    def __init__(self, name, dev, copies):
+        import torch
+        from indexed_sparse_attention_relu_b200 import binding as B
+        from indexed_sparse_attention_relu_b200 import device as DV
+        from indexed_sparse_attention_relu_b200 import workloads as W
+        self.B = B
+        self.wl = wl = W.make(name, with_caches=False)
+        self.dev = dev
+        base = DV.to_device(wl, dev)
+        self.copies = [base]
+        for _ in range(copies - 1):
+            self.copies.append(DV.DeviceWorkload(wl, base.batch, base.q_idx.clone(), base.w.clone(),
+                                                 base.k_cache.clone(),
+                                                 None if base.k_scale is None else base.k_scale.clone(), None,
+                                                 base.q.clone(), base.kv.clone()))
+        T, K = wl.T, wl.K
+        self.outs = [torch.empty((T, wl.H, wl.dc), dtype=torch.bfloat16, device=dev) for _ in self.copies]
+        self.lses = [torch.empty((T, wl.H), dtype=torch.float32, device=dev) for _ in self.copies]
+        self.ws_bytes = B.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, base.batch, K)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.idx_in = [c.indexer_in() for c in self.copies]
+        self.mla_in = [c.mla_in() for c in self.copies]
+        self.resident_bytes = sum(c.kv.numel() * 2 + c.k_cache.numel() * c.k_cache.element_size() + c.q.numel() * 2
+                                  for c in self.copies)
+
+    def step(self, i, stream, events=None):
+        j = i % len(self.copies)
+        self.B.dsa_fused_decode(self.copies[j].batch, self.idx_in[j], self.mla_in[j], self.wl.K, self.outs[j],
+                                self.lses[j], None, self.ws, self.ws_bytes, stage_events=events, stream=stream)
+
+
+def time_steps(run, steps, warmup, stream, dev, dist=None, eager=False):
+    """W warm-up steps, then K steps captured once as a CUDA graph and replayed
+    (host launch overhead cannot hide in the device time), bracketed by a
+    barrier and a device synchronize, timed with CUDA events on the launch
+    stream. Returns (total_ms, clock summary, timing mode, device status)."""
+    import torch
+    for i in range(warmup):
+        run.step(i, stream)
+    torch.cuda.synchronize(dev)
+    status = run.B.dsa_read_device_status(stream)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    for e in (t_start, t_end):
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    graph, mode = None, "eager"
+    if not eager:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream(dev)
+            with torch.cuda.graph(graph, stream=cap):
+                for i in range(steps):
+                    run.step(i, cap)
+            mode = "cuda_graph"
+        except Exception as e:
+            graph, mode = None, f"eager (graph capture failed: {type(e).__name__})"
+            torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clocks:
+        clocks.mark("start")
+        t_start.record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(steps):
+                run.step(i, stream)
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        clocks.mark("end")
+    if dist is not None:
+        dist.barrier()
+    del graph
+    return t_start.elapsed_time(t_end), clocks.summary(), mode, status
+
+
+def stage_times(run, steps, stream, dev):
+    """Per-kernel durations: eager launches with an event recorded on the launch
+    stream right before and after each stage (an event between two kernels
+    turns the programmatic launch off on that edge, and the gaps include host
+    launch latency, so these slightly overstate the in-graph stage times)."""
+    import torch
+    ev = _stage_events(run.B, steps)
+    for row in ev:
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        run.step(i, stream, ev[i])
+    torch.cuda.synchronize(dev)
+    return {
+        "indexer": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+        "topk": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+        "sparse_mla": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
+    }
+
+
+def e2e_pipelined(run, steps, warmup, dev):
+    """End to end through the public call with host buffers: every step copies
+    its inputs (q_I, w, q) from pinned host memory to the device and its output
+    back to pinned host memory. Copies run on their own streams, double
+    buffered, so step i+1's upload and step i-1's download overlap step i's
+    kernels; the timed region runs from the first upload to the last download."""
+    import torch
+    wl = run.wl
+    base = run.copies[0]
+    h_in = [(base.q_idx.cpu().pin_memory(), base.w.cpu().pin_memory(), base.q.cpu().pin_memory()) for _ in range(2)]
+    h_out = [torch.empty(run.outs[0].shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    s_in, s_run, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nb = min(2, len(run.copies))
+    in_done = [torch.cuda.Event() for _ in range(nb)]
+    run_done = [torch.cuda.Event() for _ in range(nb)]
+    out_done = [torch.cuda.Event() for _ in range(nb)]
+    h2d = sum(t.numel() * t.element_size() for t in h_in[0])
+    d2h = h_out[0].numel() * 2
+
+    def one(i):
+        j = i % nb
+        c = run.copies[j]
+        with torch.cuda.stream(s_in):
+            if i >= nb:
+                s_in.wait_event(run_done[j])          # the kernels of step i - nb no longer read buffer j
+            for dst, src in zip((c.q_idx, c.w, c.q), h_in[j]):
+                dst.copy_(src, non_blocking=True)
+            in_done[j].record(s_in)
+        s_run.wait_event(in_done[j])
+        if i >= nb:
+            s_run.wait_event(out_done[j])             # the download of step i - nb has read out[j]
+        run.B.dsa_fused_decode(c.batch, run.idx_in[j], run.mla_in[j], wl.K, run.outs[j], run.lses[j], None, run.ws,
+                               run.ws_bytes, stream=s_run)
+        run_done[j].record(s_run)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(run_done[j])
+            h_out[j].copy_(run.outs[j], non_blocking=True)
+            out_done[j].record(s_out)
+
+    for i in range(max(3, warmup)):
+        one(i)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    for i in range(steps):
+        one(i)
+    s_out.wait_event(out_done[(steps - 1) % nb])
+    e1.record(s_out)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def extra_block(name, args, dev, stream):
+    """One graph-timed measurement of another workload, with its roofline."""
+    import torch
+    t0 = time.time()
+    steps = args.extra_steps_decode if name == "c3" else args.extra_steps_prefill
+    run = Runner(name, dev, copies=2)
+    wl = run.wl
+    total_ms, clocks, mode, status = time_steps(run, steps, 2, stream, dev)
+    stages = stage_times(run, min(steps, 3), stream, dev)
+    ms = total_ms / steps
+    n_sel = int(np.minimum(wl.n_valid(), wl.K).sum())
+    block = {"name": name, "workload": WORKLOAD_TEXT[name], "steps": steps, "warmup": 2, "ms_per_step": ms,
+             "query_tokens_per_s": wl.T / (ms * 1e-3), "stage_ms": stages, "clocks": clocks, "timing": mode,
+             "device_status": [status, run.B.dsa_read_device_status(stream)],
+             "l2": f"2 rotating input copies ({run.resident_bytes / 1e9:.2f} GB) > 126 MB L2"}
+    if name == "c3":
+        peak, kind = _peaks()
+        b = algorithmic_bytes(wl, n_sel)["step"]
+        block["roofline"] = {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                             "frac": b / (ms * 1e-3) / 1e9 / peak, "peak_kind": kind, "algorithmic_bytes": b,
+                             "frac_of_8TBps": b / (ms * 1e-3) / 1e9 / 8000.0}
+    else:
+        burst, sustained, kind = _peak_tflops()
+        f = algorithmic_flops(wl, n_sel)
+        ach = f["step"] / (ms * 1e-3) / 1e12
+        block["roofline"] = {"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": sustained,
+                             "frac": ach / sustained, "peak_kind": f"{kind} sustained bf16",
+                             "frac_of_burst": ach / burst, "burst_peak": burst, "frac_of_nominal_2250": ach / 2250.0,
+                             "algorithmic_flops": f["step"],
+                             "stage_tflops": {k: f[k] / (stages[k] * 1e-3) / 1e12 for k in ("indexer", "sparse_mla")}}
+    block["setup_s"] = round(time.time() - t0 - total_ms / 1e3, 1)
+    del run
+    torch.cuda.empty_cache()
+    return block
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -198,6 +435,10 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=1, help="query tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph")
+    ap.add_argument("--extra", default="c3,c4,c5",
+                    help="comma-separated extra workloads measured after the headline (single GPU only; '' for none)")
+    ap.add_argument("--extra-steps-decode", type=int, default=20)
+    ap.add_argument("--extra-steps-prefill", type=int, default=3)
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -212,9 +453,7 @@ def main():
     import torch.distributed as dist
     from indexed_sparse_attention_relu_b200 import binding as B
     from indexed_sparse_attention_relu_b200 import build as build_mod
-    from indexed_sparse_attention_relu_b200 import device as DV
     from indexed_sparse_attention_relu_b200 import multi
-    from indexed_sparse_attention_relu_b200 import workloads as W
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU")
@@ -226,119 +465,19 @@ def main():
     build_mod.build()
     B.load()
 
-    # ---- inputs: one workload, cloned into rotating copies on the device
-    wl = W.make(args.config, with_caches=False)
-    base = DV.to_device(wl, dev)
-    copies = [base]
-    for _ in range(args.copies - 1):
-        c = DV.DeviceWorkload(wl, base.batch, base.q_idx.clone(), base.w.clone(), base.k_cache.clone(),
-                              None if base.k_scale is None else base.k_scale.clone(), None, base.q.clone(),
-                              base.kv.clone())
-        copies.append(c)
+    run = Runner(args.config, dev, args.copies)
+    wl = run.wl
     T, K = wl.T, wl.K
     stream = torch.cuda.current_stream(dev)
-    outs = [torch.empty((T, wl.H, wl.dc), dtype=torch.bfloat16, device=dev) for _ in copies]
-    lses = [torch.empty((T, wl.H), dtype=torch.float32, device=dev) for _ in copies]
-    ws_bytes = B.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, base.batch, K)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    idx_in = [c.indexer_in() for c in copies]
-    mla_in = [c.mla_in() for c in copies]
-
-    def step(i, events=None, st=None):
-        j = i % len(copies)
-        B.dsa_fused_decode(copies[j].batch, idx_in[j], mla_in[j], K, outs[j], lses[j], None, ws, ws_bytes,
-                           stage_events=events, stream=stream if st is None else st)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(dev)
-    status = B.dsa_read_device_status(stream)
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    for e in [x for row in ev for x in row] + [t_start, t_end]:
-        e.record(stream)            # creates the CUDA events outside the timed region
-    torch.cuda.synchronize(dev)
-    # The K timed steps are captured once as one CUDA graph and replayed once,
-    # so host launch overhead cannot hide in the device time (every call of
-    # the library is capture-safe: no allocation, no synchronisation).
-    graph = None
-    timing_mode = "eager"
-    if not args.eager:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            cap = torch.cuda.Stream(dev)
-            with torch.cuda.graph(graph, stream=cap):
-                for i in range(args.steps):
-                    step(i, None, st=cap)
-            timing_mode = "cuda_graph"
-        except Exception as e:  # report and fall back to eager launches
-            graph = None
-            timing_mode = f"eager (graph capture failed: {type(e).__name__})"
-            torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    # timed region: K steps exactly as a caller runs them (programmatic launch
-    # between the kernels, no events in between)
-    with ClockSampler(dev) as clocks:
-        t_start.record(stream)
-        if graph is not None:
-            graph.replay()
-        else:
-            for i in range(args.steps):
-                step(i)
-        t_end.record(stream)
-        torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    # per-kernel durations: a second pass of K steps, launched eagerly with an
-    # event recorded on the launch stream right before and after each stage
-    # (events inside a graph cannot be timed; an event between two kernels also
-    # turns the programmatic launch off on that edge)
-    for i in range(args.steps):
-        step(i, ev[i])
-    torch.cuda.synchronize(dev)
-    stage_ms = {
-        "indexer": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
-        "topk": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
-        "sparse_mla": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
-    }
+    total_ms, clocks, timing_mode, status = time_steps(run, args.steps, args.warmup, stream, dev,
+                                                      dist if world > 1 else None, eager=args.eager)
+    stage_ms = stage_times(run, args.steps, stream, dev)
     # the job's time is its slowest rank's; every rank ran its own T queries
     total_ms = multi.max_over_ranks(total_ms, dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
     value = multi.job_throughput([T] * world, ms_per_step)
 
-    # ---- end to end through the C ABI with host buffers (pinned), copies timed
-    h_qidx = base.q_idx.cpu().pin_memory()
-    h_w = base.w.cpu().pin_memory()
-    h_q = base.q.cpu().pin_memory()
-    h_out = torch.empty(outs[0].shape, dtype=torch.bfloat16).pin_memory()
-    h2d = h_qidx.numel() * 2 + h_w.numel() * 4 + h_q.numel() * 2
-    d2h = h_out.numel() * 2
-
-    def e2e_step(i):
-        j = i % len(copies)
-        c = copies[j]
-        c.q_idx.copy_(h_qidx, non_blocking=True)
-        c.w.copy_(h_w, non_blocking=True)
-        c.q.copy_(h_q, non_blocking=True)
-        B.dsa_fused_decode(c.batch, idx_in[j], mla_in[j], K, outs[j], lses[j], None, ws, ws_bytes, stream=stream)
-        h_out.copy_(outs[j], non_blocking=True)
-
-    for i in range(max(3, args.warmup)):
-        e2e_step(i)
-    torch.cuda.synchronize(dev)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.steps
+    e2e_ms, h2d, d2h = e2e_pipelined(run, args.steps, args.warmup, dev)
     e2e_ms = multi.max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
     status2 = B.dsa_read_device_status(stream)
 
@@ -376,8 +515,7 @@ def main():
         "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config, "B": wl.B, "L_max": wl.Lmax,
                    "T": T, "K": K, "H_I": wl.HI, "d_I": wl.dI, "H": wl.H, "d_c": wl.dc, "d_rope": wl.dr,
                    "index_keys": wl.key_dtype, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"{len(copies)} rotating input copies "
-                         f"({len(copies) * (base.kv.numel() * 2 + base.k_cache.numel() * base.k_cache.element_size()) / 1e9:.2f} GB) > 126 MB L2"},
+                   "l2": f"{len(run.copies)} rotating input copies ({run.resident_bytes / 1e9:.2f} GB) > 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
                      "algorithmic_bytes": algo[dom], "avg_launch_ms": stage_ms[dom]},
@@ -386,18 +524,28 @@ def main():
                           "algorithmic_bytes": algo["step"]},
         "stage_ms": stage_ms,
         "stage_ms_note": "second K-step pass, eager launches with CUDA events between the stages",
-        "clocks": clocks.summary(),
+        "clocks": clocks,
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "note": "pinned host buffers; uploads and downloads on their own streams, double buffered"},
         "gpu_launches": launches_per_step * args.steps,
         "timing": timing_mode,
         "device_status": [status, status2],
     }
+    del run
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n, dt, thr = run_cpu_oracle(wl, args.cpu_tokens, min_seconds=args.cpu_seconds)
         line["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
                                 "sample": f"{min(args.cpu_tokens, wl.T)} query tokens of the same workload (full "
                                           f"causal history), fp64, repeated to {n} tokens in {dt:.1f} s"}
+    if world == 1 and args.extra:
+        line["configs"] = []
+        for name in [x for x in args.extra.split(",") if x and x != args.config]:
+            try:
+                line["configs"].append(extra_block(name, args, dev, stream))
+            except Exception as e:  # report, keep the headline
+                line["configs"].append({"name": name, "error": f"{type(e).__name__}: {e}"})
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

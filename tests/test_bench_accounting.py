@@ -40,3 +40,21 @@ def test_cpu_baseline_repeats_until_the_minimum_time():
     wl = W.make("c1", with_caches=False)
     n, dt, thr = bench.run_cpu_oracle(wl, 2, min_seconds=0.2)
     assert dt >= 0.2 and n % 2 == 0 and n >= 2 and thr >= 1
+
+
+def test_prefill_flops_by_hand():
+    """Causal prefill of 32768 tokens: the indexer scores every causal pair
+    (sum_{t<32768} (t+1) pairs) at 64 heads x 128 dims, and the attention runs
+    QK^T over 576 dims and PV over 512 dims for min(t+1, 2048) selected rows
+    per token at 128 heads. (Shapes only: the query tensors are not drawn.)"""
+    import types
+    nv = np.arange(1, 32769, dtype=np.int32)
+    wl = types.SimpleNamespace(HI=64, dI=128, H=128, D=576, dc=512, K=2048, n_valid=lambda: nv)
+    n_sel = int(np.minimum(nv, 2048).sum())
+    pairs = 32768 * 32769 // 2
+    sel = 2048 * 2049 // 2 + (32768 - 2048) * 2048
+    assert (pairs, n_sel) == (536887296, sel) and sel == 65012736
+    f = bench.algorithmic_flops(wl, n_sel)
+    assert f["indexer"] == pairs * 64 * 128 * 2 == 8796361457664
+    assert f["sparse_mla"] == sel * 128 * (576 + 512) * 2 == 18107867332608
+    assert f["step"] == f["indexer"] + f["sparse_mla"]
