@@ -203,11 +203,13 @@ def _cache(seed, tag, B, Lmax, lens, dim, law, rows_needed=None):
 
 
 def make(name: str, *, with_caches: bool = True, rows_needed: Optional[Dict[int, list]] = None,
-         tokens: Optional[slice] = None) -> Workload:
+         tokens: Optional[slice] = None, queries: bool = True) -> Workload:
     """Build the synthetic workload ``name`` (see the module docstring).
 
     ``with_caches=False`` skips drawing the two caches (k_idx, kv).
     ``rows_needed`` limits cache generation to the blocks holding those rows.
+    ``queries=False`` skips drawing the query tensors too (shapes and laws
+    only: q_idx, w and q are left empty).
     """
     seed = _SEEDS[name]
     if name == "c1":
@@ -262,9 +264,14 @@ def make(name: str, *, with_caches: bool = True, rows_needed: Optional[Dict[int,
 
     T = int(cu_q[-1])
     D = dc + dr
-    q_idx = bf16_round(_draw_rows(seed, "q_idx", T, HI * dI, law_q)).reshape(T, HI, dI)
-    w = _draw_rows(seed, "w", T, HI, law_w).astype(np.float32)
-    q = bf16_round(_draw_rows(seed, "q", T, H * D, law_mla)).reshape(T, H, D)
+    if queries:
+        q_idx = bf16_round(_draw_rows(seed, "q_idx", T, HI * dI, law_q)).reshape(T, HI, dI)
+        w = _draw_rows(seed, "w", T, HI, law_w).astype(np.float32)
+        q = bf16_round(_draw_rows(seed, "q", T, H * D, law_mla)).reshape(T, H, D)
+    else:
+        q_idx = np.zeros((0, HI, dI), np.float32)
+        w = np.zeros((0, HI), np.float32)
+        q = np.zeros((0, H, D), np.float32)
     k_idx = kv = None
     if with_caches:
         k_idx = _cache(seed, "k_idx", B, Lmax, lens, dI, law_k, rows_needed)
@@ -296,7 +303,7 @@ def scaled(name: str, *, B: int, Lmax: int, T_per_seq: int = 1, lens=None, K: Op
     Used by the parity tests: sizes the oracle finishes in seconds that still
     span several tiles and a ragged tail. Queries are the last ``T_per_seq``
     positions of every sequence."""
-    base = make(name, with_caches=False, tokens=slice(0, 1))
+    base = make(name, with_caches=False, queries=False)
     HI = base.HI if HI is None else HI
     dI = base.dI if dI is None else dI
     H = base.H if H is None else H

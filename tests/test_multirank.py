@@ -105,3 +105,105 @@ def test_two_gloo_ranks_agree():
 
 def test_max_over_ranks_without_group_is_identity():
     assert multi.max_over_ranks(2.5) == 2.5
+
+
+# ----------------------------------------------------------------------------- zigzag context parallelism
+
+def test_zigzag_matches_the_pages_examples():
+    """The pages' two worked assignments: with 2 cards and 4 segments, card 0
+    takes segments 1 and 4 and card 1 segments 2 and 3 (1-based); with 8
+    devices... device 0 of a sequence of length L cut for 4 devices handles
+    [0, L/8) and [7L/8, L)."""
+    L = 4096
+    two = multi.zigzag_segments(L, 2)
+    seg = [(0, 1024), (1024, 2048), (2048, 3072), (3072, 4096)]
+    assert two == [[seg[0], seg[3]], [seg[1], seg[2]]]
+    four = multi.zigzag_segments(L, 4)
+    assert four[0] == [(0, L // 8), (7 * L // 8, L)]
+
+
+def test_zigzag_balances_causal_work():
+    """Equal segments paired early-with-late give every rank the same causal
+    work; a contiguous split gives the last rank 2N-1 times the first's."""
+    T = 32768
+    for world in (2, 4, 8):
+        loads = [multi.causal_work(multi.zigzag_rows(T, world, d)) for d in range(world)]
+        assert max(loads) == min(loads)
+        assert sum(loads) == T * (T + 1) // 2
+        contiguous = [multi.causal_work(np.arange(d * T // world, (d + 1) * T // world)) for d in range(world)]
+        assert max(contiguous) / min(contiguous) > 2 * world - 1.5
+    # uneven segment sizes (T not a multiple of 2N): within one segment's worth of rows
+    T = 1001
+    loads = [multi.causal_work(multi.zigzag_rows(T, 3, d)) for d in range(3)]
+    assert max(loads) - min(loads) <= 2 * T
+
+
+def test_zigzag_restore_is_the_inverse():
+    rng = np.random.default_rng(5)
+    for T, world in ((17, 2), (1000, 4), (64, 8), (3, 2)):
+        data = rng.standard_normal((T, 3))
+        parts = [data[multi.zigzag_rows(T, world, d)] for d in range(world)]
+        assert np.array_equal(multi.zigzag_restore(parts, T, world), data)
+        flat = np.sort(np.concatenate([multi.zigzag_rows(T, world, d) for d in range(world)]))
+        assert np.array_equal(flat, np.arange(T))
+
+
+def _cp_rank_main(rank, world, port, q):
+    """One rank of a context-parallel prefill: it takes its zigzag rows, holds
+    the cache rows of its own segments, all-gathers everyone's rows into the
+    full caches, runs the whole path (the fp64 oracle stands in for the
+    kernels on CPU) for its rows, and all-gathers the results."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import dataclasses
+    import datetime
+
+    import oracle
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        wl = W.scaled("c4", B=1, Lmax=96, T_per_seq=96, K=16, HI=4, dI=32, H=4, dc=64, dr=16)
+        rows = multi.zigzag_rows(wl.T, world, rank)
+        # this rank's cache rows (positions = its query rows in a prefill)
+        k_mine = torch.from_numpy(wl.k_idx[0, rows])
+        kv_mine = torch.from_numpy(wl.kv[0, rows])
+        pos_mine = torch.from_numpy(rows)
+        k_all = multi.all_gather_rows(k_mine, dist)
+        kv_all = multi.all_gather_rows(kv_mine, dist)
+        pos_all = multi.all_gather_rows(pos_mine, dist)
+        k_full = np.zeros_like(wl.k_idx)
+        kv_full = np.zeros_like(wl.kv)
+        for p, k, v in zip(pos_all, k_all, kv_all):
+            k_full[0, p.numpy()] = k.numpy()
+            kv_full[0, p.numpy()] = v.numpy()
+        local = dataclasses.replace(wl, k_idx=k_full, kv=kv_full)
+        _, idx, out, lse = oracle.dsa(local, rows)
+        idx_all = multi.all_gather_rows(torch.from_numpy(idx), dist)
+        out_all = multi.all_gather_rows(torch.from_numpy(out), dist)
+        q.put((rank, [t.numpy() for t in idx_all], [t.numpy() for t in out_all]))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_zigzag_context_parallel_prefill_two_gloo_ranks():
+    """Two ranks reproduce the single-process result exactly once the zigzag
+    shards are gathered and put back in order."""
+    import oracle
+
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q.get(timeout=180) for _ in range(world)], key=lambda g: g[0])
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    wl = W.scaled("c4", B=1, Lmax=96, T_per_seq=96, K=16, HI=4, dI=32, H=4, dc=64, dr=16)
+    _, want_idx, want_out, _ = oracle.dsa(wl)
+    for _, idx_parts, out_parts in got:           # every rank holds the whole result
+        assert np.array_equal(multi.zigzag_restore(idx_parts, wl.T, world), want_idx)
+        assert np.array_equal(multi.zigzag_restore(out_parts, wl.T, world), want_out)
