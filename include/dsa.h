@@ -91,9 +91,26 @@ typedef enum {
  *   q_pos    [T]   int32 device: position of each query token inside its
  *                  sequence; its causal history is s <= q_pos.
  *   seq_lens [B]   int32 device: valid cache rows of sequence b (<= max_seq_len).
- *   max_seq_len    L_max, the row stride of the caches: sequence b's rows are
- *                  cache[b * L_max + s].
- *   block_table / page_size: reserved for paged caches; must be NULL / 0.
+ *   max_seq_len    L_max: the longest sequence the caches hold, and the row
+ *                  stride of the score rows. Contiguous caches (block_table
+ *                  NULL): sequence b's row s is cache row b * L_max + s.
+ *   block_table    [B, max_pages] int32 device, or NULL. Paged caches (the
+ *                  fused indexer reading the paged key cache directly:
+ *                  section 3 of "Optimizing Inference for New Model
+ *                  Architectures ..."): every cache -- index keys, their FP8
+ *                  scales and the latent KV rows -- is a pool of num_pages
+ *                  pages of page_size rows, all under this one table, and
+ *                  sequence b's row s is pool row
+ *                    block_table[b * max_pages + s / page_size] * page_size
+ *                      + s % page_size,
+ *                  max_pages = ceil(max_seq_len / page_size). Only the
+ *                  entries of pages that hold rows s < seq_lens[b] are read.
+ *                  An entry outside [0, num_pages) is never dereferenced: the
+ *                  row reads as pool row 0 and DSA_ERR_DEVICE_INDEX is set.
+ *                  Positions (scores, indices) stay logical.
+ *   page_size      rows per page, a positive multiple of 64 (paged), else 0.
+ *   num_pages      pages in the pool (paged), else 0; num_pages * page_size
+ *                  must be below 2^31.
  * A query's candidate count is n_valid(t) = min(q_pos[t] + 1, seq_lens[b]). */
 typedef struct {
     int32_t batch;
@@ -104,13 +121,15 @@ typedef struct {
     const int32_t *seq_lens;
     const int32_t *block_table;
     int32_t page_size;
+    int32_t num_pages;
 } dsa_batch;
 
 /* Lightning Indexer inputs.
  *   q        bf16 [T, n_heads, head_dim]       indexer queries q_I
  *   w        fp32 [T, n_heads]                 head weights
- *   k_cache  [B, L_max, head_dim]              index keys, bf16 or e4m3 codes
- *   k_scale  fp32 [B, L_max, head_dim/scale_group] per-group scales (FP8 only;
+ *   k_cache  [rows, head_dim]                  index keys, bf16 or e4m3 codes;
+ *            rows = B * L_max (contiguous) or num_pages * page_size (paged)
+ *   k_scale  fp32 [rows, head_dim/scale_group] per-group scales (FP8 only;
  *            the key value is decode(code) * scale), NULL for BF16
  *   scale_group: elements per scale; must equal head_dim for the FP8 indexer. */
 typedef struct {
@@ -126,7 +145,8 @@ typedef struct {
 
 /* Sparse MLA inputs.
  *   q   bf16 [T, n_heads, d_latent + d_rope]
- *   kv  bf16 [B, L_max, d_latent + d_rope]   latent rows; value = first d_latent
+ *   kv  bf16 [rows, d_latent + d_rope]   latent rows (rows as for k_cache);
+ *       value = first d_latent
  *   softmax_scale: multiplies q . kv before the softmax. */
 typedef struct {
     int32_t n_heads;

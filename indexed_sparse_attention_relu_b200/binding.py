@@ -57,7 +57,7 @@ class DsaError(RuntimeError):
 class dsa_batch(ctypes.Structure):
     _fields_ = [("batch", c_int32), ("num_q", c_int32), ("max_seq_len", c_int32),
                 ("cu_q", c_void_p), ("q_pos", c_void_p), ("seq_lens", c_void_p),
-                ("block_table", c_void_p), ("page_size", c_int32)]
+                ("block_table", c_void_p), ("page_size", c_int32), ("num_pages", c_int32)]
 
 
 class dsa_indexer_in(ctypes.Structure):
@@ -140,12 +140,15 @@ def _stream(stream) -> int | None:
 # ----------------------------------------------------------------------------- struct builders
 
 class Batch:
-    """Owns the int32 metadata tensors and exposes the dsa_batch struct."""
+    """Owns the int32 metadata tensors and exposes the dsa_batch struct.
+    ``block_table`` ([B, ceil(max_seq_len / page_size)] int32), ``page_size``
+    and ``num_pages`` describe paged caches; all None/0 for contiguous ones."""
 
-    def __init__(self, cu_q: torch.Tensor, q_pos: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int):
-        self.cu_q, self.q_pos, self.seq_lens = cu_q, q_pos, seq_lens
+    def __init__(self, cu_q: torch.Tensor, q_pos: torch.Tensor, seq_lens: torch.Tensor, max_seq_len: int,
+                 block_table: torch.Tensor | None = None, page_size: int = 0, num_pages: int = 0):
+        self.cu_q, self.q_pos, self.seq_lens, self.block_table = cu_q, q_pos, seq_lens, block_table
         self.struct = dsa_batch(seq_lens.numel(), q_pos.numel(), int(max_seq_len), _ptr(cu_q), _ptr(q_pos),
-                                _ptr(seq_lens), None, 0)
+                                _ptr(seq_lens), _ptr(block_table), int(page_size), int(num_pages))
 
     @property
     def ref(self):

@@ -10,6 +10,7 @@
 
 #include "dsa_common.cuh"
 #include "indexer.cuh"
+#include "indexer_decode.cuh"
 #include "quant.cuh"
 #include "sparse_mla.cuh"
 #include "sparse_mla_pipe.cuh"
@@ -64,7 +65,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D map over the index-key cache: x = element within a key, y = key row.
-dsa_status make_key_map(CUtensorMap* map, const void* base, int64_t rows, int din, bool fp8) {
+// Boxes of 128 key rows (one tile), or 64 for paged caches (a tile is then
+// two boxes, each inside one page).
+dsa_status make_key_map(CUtensorMap* map, const void* base, int64_t rows, int din, bool fp8, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(din), static_cast<cuuint64_t>(rows)};
@@ -72,12 +75,12 @@ dsa_status make_key_map(CUtensorMap* map, const void* base, int64_t rows, int di
   const cuuint32_t estr[2] = {1, 1};
   CUresult r;
   if (fp8) {
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(din), 128};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(din), static_cast<cuuint32_t>(box_rows)};
     r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   } else {
-    const cuuint32_t box[2] = {64, 128};  // one 128-byte swizzle atom column of 128 keys
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};  // one 128-byte swizzle atom column
     r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -110,12 +113,40 @@ dsa_status check_batch(const dsa_batch* bt) {
                 bt->num_q, bt->max_seq_len);
   if (bt->num_q > 0 && (!bt->cu_q || !bt->q_pos || !bt->seq_lens))
     return fail(DSA_ERR_INVALID_ARGUMENT, "cu_q, q_pos and seq_lens must be non-NULL");
-  if (bt->block_table || bt->page_size)
-    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "paged caches (block_table) are not supported");
   if (static_cast<int64_t>(bt->batch) * bt->max_seq_len >= (int64_t(1) << 31))
     return fail(DSA_ERR_UNSUPPORTED_SHAPE, "batch * max_seq_len must be < 2^31");
+  if (!bt->block_table) {
+    if (bt->page_size != 0 || bt->num_pages != 0)
+      return fail(DSA_ERR_INVALID_ARGUMENT, "page_size and num_pages must be 0 without a block table");
+    return DSA_OK;
+  }
+  if (bt->page_size <= 0 || bt->page_size % 64 != 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "page_size %d must be a positive multiple of 64", bt->page_size);
+  if (bt->num_pages <= 0) return fail(DSA_ERR_INVALID_ARGUMENT, "num_pages %d must be positive", bt->num_pages);
+  if (static_cast<int64_t>(bt->num_pages) * bt->page_size >= (int64_t(1) << 31))
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "num_pages * page_size must be < 2^31");
+  if (reinterpret_cast<uintptr_t>(bt->block_table) & 3u)
+    return fail(DSA_ERR_MISALIGNED, "block_table must be 4-byte aligned");
   return DSA_OK;
 }
+
+// Rows of every cache: B * L_max (contiguous) or the page pool.
+int64_t cache_rows(const dsa_batch* bt) {
+  return bt->block_table ? static_cast<int64_t>(bt->num_pages) * bt->page_size
+                         : static_cast<int64_t>(bt->batch) * bt->max_seq_len;
+}
+
+CacheMap cache_map(const dsa_batch* bt) {
+  CacheMap m;
+  m.table = bt->block_table;
+  m.L_max = bt->max_seq_len;
+  m.page_size = bt->block_table ? bt->page_size : 0;
+  m.max_pages = bt->block_table ? (bt->max_seq_len + bt->page_size - 1) / bt->page_size : 0;
+  m.num_pages = bt->block_table ? bt->num_pages : 0;
+  return m;
+}
+
+int key_box_rows(const dsa_batch* bt) { return bt->block_table ? 64 : 128; }
 
 dsa_status check_indexer(const dsa_batch* bt, const dsa_indexer_in* in) {
   if (!in) return fail(DSA_ERR_INVALID_ARGUMENT, "indexer input is NULL");
@@ -267,7 +298,7 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
                             cudaStream_t st, bool pdl) {
   using C = IndexerCfg<HI, DIN, G, FP8>;
   CUtensorMap map;
-  dsa_status s = make_key_map(&map, in->k_cache, static_cast<int64_t>(bt->batch) * bt->max_seq_len, DIN, FP8);
+  dsa_status s = make_key_map(&map, in->k_cache, cache_rows(bt), DIN, FP8, key_box_rows(bt));
   if (s != DSA_OK) return s;
   auto kern = indexer_scores_kernel<HI, DIN, G, FP8>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
@@ -296,6 +327,7 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   p.seq_lens = bt->seq_lens;
   p.B = bt->batch;
   p.L_max = bt->max_seq_len;
+  p.cm = cache_map(bt);
   p.q = static_cast<const __nv_bfloat16*>(in->q);
   p.w = in->w;
   p.k_scale = in->k_scale;
@@ -317,10 +349,53 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   return check_launch("indexer_scores");
 }
 
+// One query token per group (decode): one CTA per SM, each taking an equal
+// range of the flattened key-tile list of all tokens.
+template <int HI, int DIN, bool FP8>
+dsa_status launch_indexer_decode(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
+                                 cudaStream_t st, bool pdl) {
+  using C = IdxDecCfg<HI, DIN, FP8>;
+  CUtensorMap kmap, qmap;
+  dsa_status s = make_key_map(&kmap, in->k_cache, cache_rows(bt), DIN, FP8, key_box_rows(bt));
+  if (s != DSA_OK) return s;
+  if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(bt->num_q) * HI, DIN, HI)) != DSA_OK) return s;
+  auto kern = indexer_decode_kernel<HI, DIN, FP8>;
+  if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
+  IdxDecParams p;
+  p.cu_q = bt->cu_q;
+  p.q_pos = bt->q_pos;
+  p.seq_lens = bt->seq_lens;
+  p.k_scale = FP8 ? in->k_scale : nullptr;
+  p.B = bt->batch;
+  p.T = bt->num_q;
+  p.L_max = bt->max_seq_len;
+  p.cm = cache_map(bt);
+  p.scores = scores;
+  p.ld = ld;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, kmap, qmap, in->w, p);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "indexer (decode) launch: %s", cudaGetErrorString(e));
+  return check_launch("indexer_scores (decode)");
+}
+
 template <int HI, int DIN>
 dsa_status launch_indexer_g(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
                             cudaStream_t st, bool pdl) {
   const bool fp8 = in->key_dtype == DSA_KEY_FP8_E4M3;
+  // decode (one token per group): the balanced one-CTA-per-SM kernel while a
+  // CTA's segment list (at most one entry per token) fits
+  if (indexer_group(bt) == 1 && bt->num_q <= IdxDecCfg<HI, DIN, false>::MAXSEG)
+    return fp8 ? launch_indexer_decode<HI, DIN, true>(bt, in, scores, ld, st, pdl)
+               : launch_indexer_decode<HI, DIN, false>(bt, in, scores, ld, st, pdl);
   if (indexer_group(bt) == 4)
     return fp8 ? launch_indexer_t<HI, DIN, 4, true>(bt, in, scores, ld, st, pdl)
                : launch_indexer_t<HI, DIN, 4, false>(bt, in, scores, ld, st, pdl);
@@ -418,6 +493,7 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   p.seq_lens = bt->seq_lens;
   p.B = bt->batch;
   p.L_max = bt->max_seq_len;
+  p.cm = cache_map(bt);
   p.T = T;
   p.H = H;
   p.K = k;
@@ -508,13 +584,14 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
   if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   CUtensorMap qmap, kvmap;
   if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(T) * C::M, C::D, C::M)) != DSA_OK) return s;
-  if ((s = make_bf16_rows_map(&kvmap, in->kv, static_cast<int64_t>(bt->batch) * bt->max_seq_len, C::D, 1)) != DSA_OK)
+  if ((s = make_bf16_rows_map(&kvmap, in->kv, cache_rows(bt), C::D, 1)) != DSA_OK)
     return s;
   PipeParams p;
   p.cu_q = bt->cu_q;
   p.seq_lens = bt->seq_lens;
   p.B = bt->batch;
   p.L_max = bt->max_seq_len;
+  p.cm = cache_map(bt);
   p.T = T;
   p.K = k;
   p.idx = idx;

@@ -40,6 +40,41 @@ __device__ uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 // (set by dsa_debug_withhold_signal(); 0 in normal operation).
 __device__ int g_debug_withhold = 0;
 
+// ---------------------------------------------------------------- cache rows
+// Where logical row s of sequence b lives in a cache (index keys, their FP8
+// scales and the latent KV rows all share it). Contiguous caches: row
+// b * L_max + s. Paged caches (block table; the paged key cache the fused
+// indexer reads, section 3 of "Optimizing Inference for New Model
+// Architectures ..."): a pool of num_pages pages of page_size rows, and row
+// table[b * max_pages + s / page_size] * page_size + s % page_size. A page id
+// outside [0, num_pages) is never dereferenced: row() reports it (ok = false)
+// and returns row 0, which the caller masks.
+struct CacheMap {
+  const int32_t* table;  // [B, max_pages] or null (contiguous)
+  int32_t L_max;
+  int32_t page_size;     // multiple of 64 (paged)
+  int32_t max_pages;     // ceil(L_max / page_size)
+  int32_t num_pages;
+
+  __device__ __forceinline__ bool paged() const { return table != nullptr; }
+  __device__ __forceinline__ int32_t row(int b, int s, bool& ok) const {
+    if (table == nullptr) {
+      ok = true;
+      return b * L_max + s;
+    }
+    const int32_t pg = __ldg(table + static_cast<int64_t>(b) * max_pages + s / page_size);
+    ok = static_cast<uint32_t>(pg) < static_cast<uint32_t>(num_pages);
+    return ok ? pg * page_size + s % page_size : 0;
+  }
+  // As row(), recording a bad page id in the status word.
+  __device__ __forceinline__ int32_t row_checked(int b, int s) const {
+    bool ok;
+    const int32_t r = row(b, s, ok);
+    if (!ok) set_device_status(DSA_ERR_DEVICE_INDEX);
+    return r;
+  }
+};
+
 __device__ __forceinline__ uint64_t wait_limit_ns() {
   return *reinterpret_cast<volatile uint64_t*>(&g_wait_limit_ns);
 }

@@ -34,10 +34,11 @@ struct IndexerParams {
   int32_t L_max;
   const __nv_bfloat16* q;   // [T, HI, DIN]
   const float* w;           // [T, HI]
-  const float* k_scale;     // [B*L_max] (FP8, one scale per key) or null
+  const float* k_scale;     // one scale per cache row (FP8) or null
   float* scores;            // [T, ld]
   int64_t ld;
   int32_t tiles_per_cta;
+  CacheMap cm;              // cache rows (contiguous or paged)
 };
 
 template <int HI, int DIN, int G, bool FP8>
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
           misc[7 + i] = nv;
           nk = max(nk, nv);
         }
+        misc[12] = nk;
         const int n_tiles = (nk + 127) / 128;
         tb = blockIdx.y * p.tiles_per_cta;
         te = min(n_tiles, tb + p.tiles_per_cta);
@@ -205,6 +207,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   }
   const int t0 = misc[1];
   const int nt = misc[2];
+  const int nk = misc[12];  // causal candidates of the group's last token
   const int n_tiles = tile_end - tile_begin;
   const int64_t row0 = static_cast<int64_t>(b) * p.L_max;
 
@@ -212,15 +215,30 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
   // latency overlaps the query staging and the TMEM allocation below.
   auto issue_tile = [&](int it) {
     const int st = it % C::ST;
-    const int32_t y = static_cast<int32_t>(row0 + static_cast<int64_t>(tile_begin + it) * 128);
+    const int s0 = (tile_begin + it) * 128;  // first key position of the tile
     const uint32_t dst = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES);
-    if constexpr (FP8) {
-      mbar_arrive_expect_tx(&full[st], C::U8_TILE);
-      tma_load_2d(dst, &kmap, 0, y, &full[st]);
-    } else {
-      mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
+    mbar_arrive_expect_tx(&full[st], FP8 ? C::U8_TILE : C::TILE_BYTES);
+    if (!p.cm.paged()) {
+      const int32_t y = static_cast<int32_t>(row0 + s0);
+      if constexpr (FP8) {
+        tma_load_2d(dst, &kmap, 0, y, &full[st]);
+      } else {
 #pragma unroll
-      for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384, &kmap, a * 64, y, &full[st]);
+        for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384, &kmap, a * 64, y, &full[st]);
+      }
+    } else {
+      // paged: two 64-row boxes (a page holds a whole number of them); a half
+      // past the last candidate reloads the first half (its rows are masked)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int32_t y = p.cm.row_checked(b, (s0 + 64 * h < nk) ? s0 + 64 * h : s0);
+        if constexpr (FP8) {
+          tma_load_2d(dst + h * 64 * DIN, &kmap, 0, y, &full[st]);
+        } else {
+#pragma unroll
+          for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384 + h * 8192, &kmap, a * 64, y, &full[st]);
+        }
+      }
     }
   };
   const int prologue_tiles = min(n_tiles, C::ST);
@@ -401,7 +419,11 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
       const int64_t s = static_cast<int64_t>(tile_begin + it) * 128 + r;
       float sigma = 1.0f;
       if constexpr (FP8) {
-        if (s < p.L_max) sigma = __ldg(p.k_scale + row0 + s);
+        if (s < nk) {
+          bool ok;
+          const int32_t kr = p.cm.row(b, static_cast<int>(s), ok);
+          sigma = __ldg(p.k_scale + (p.cm.paged() ? static_cast<int64_t>(kr) : row0 + s));
+        }
       }
       if (s < p.ld) {
         constexpr int GPART = C::EPI_WARPS == 8 ? G / 2 : G;  // tokens this warp scores

@@ -59,6 +59,7 @@ struct MlaParams {
   float* lse;                // [T, H] or null
   float* part_o;             // [T, HB, splits][DC / 4][64][4] split partials (splits > 1)
   float2* part_ml;           // [T, HB, splits, 64] (running max, running sum)
+  CacheMap cm;               // cache rows (contiguous or paged)
 };
 
 template <int D, int DC>
@@ -246,7 +247,6 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     constexpr int CPR = C::DP / 8;                 // 16-byte chunks per stored row
     constexpr int ROUNDS = (C::RPW * CPR + 31) / 32;  // instructions per warp per tile
     const int pw = warp - 4;
-    const __nv_bfloat16* kv_seq = kv + static_cast<int64_t>(b) * p.L_max * D;
     auto row_index = [&](int tile) -> int {
       const int k = k_begin + tile * C::TK + C::RPW * pw + lane;
       return (lane < C::RPW && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
       if (!ok) break;
       const bool okr = cur >= 0 && cur < len;
       if (lane < C::RPW && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
-      const int mine = okr ? cur : -1;
+      const int mine = okr ? p.cm.row_checked(b, cur) : -1;  // cache row of this lane's key
       const uint32_t stage = smem_u32(smem + C::OFF_KV + sl * C::KV_BYTES);
 #pragma unroll 2
       for (int q = 0; q < ROUNDS; ++q) {
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
         if (flat < C::RPW * CPR) {
           const int r = C::RPW * pw + rl;
           const bool has = srow >= 0 && c * 8 < D;
-          const __nv_bfloat16* src = kv_seq + static_cast<int64_t>(has ? srow : 0) * D + (has ? c * 8 : 0);
+          const __nv_bfloat16* src = kv + static_cast<int64_t>(has ? srow : 0) * D + (has ? c * 8 : 0);
           cp_async_16(stage + (c >> 3) * C::ATOM_COL + sw128_offset(r, c & 7), has ? src : kv, has ? 16u : 0u);
         }
       }

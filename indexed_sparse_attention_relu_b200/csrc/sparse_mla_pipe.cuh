@@ -49,6 +49,7 @@ struct PipeParams {
   float2* fin;               // [RING_SMS, 128] final (running max, running sum) per head row
   float* part_o;             // [T, splits][512 / 4][128][4] split partials (splits > 1)
   float2* part_ml;           // [T, splits, 128]
+  CacheMap cm;               // cache rows (contiguous or paged)
 };
 
 struct PipeCfg {
@@ -385,14 +386,14 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       // thread. A leader waits for the stage and arms its barrier; the others
       // learn through a per-tile flag whether to go on, so every tile is
       // issued whole or not at all. Invalid rows (-1, or outside the
-      // sequence) fetch the sequence's row 0 instead: their logits are masked
-      // to -inf below and their P is 0.
+      // sequence) fetch the sequence's row 0 (paged caches: the pool's row 0)
+      // instead: their logits are masked to -inf below and their P is 0.
       pdl_wait_prior();  // the selected indices (Top-K output) are complete from here on
       const int gl = threadIdx.x - 4 * 32;  // 0 .. 32 * NGATHER - 1
       const bool leader = gl == 0;
       const bool active = gl < 16 * 9;
       const int g = gl / 9, a = gl - (gl / 9) * 9;
-      const int32_t row0 = b * p.L_max;
+      const int32_t row0 = p.cm.paged() ? 0 : b * p.L_max;  // stand-in row for invalid keys
       {
         // stage this split's indices (eight independent loads in flight per thread)
         const int nk = k_end - k_begin;
@@ -437,7 +438,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           for (int i = 0; i < 4; ++i) {
             const bool v = cur[i] >= 0 && cur[i] < len;
             if (a == 0 && cur[i] != -1 && !v) set_device_status(DSA_ERR_DEVICE_INDEX);
-            y[i] = row0 + (v ? cur[i] : 0);
+            y[i] = v ? p.cm.row_checked(b, cur[i]) : row0;
           }
           tma_gather4(smem_u32(smem + C::A_OFF_K + sl * C::K_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0], y[1],
                       y[2], y[3], &kv_full[sl]);
@@ -548,7 +549,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       const bool leader = gl == 0;
       const bool active = gl < 16 * 8;
       const int g = gl >> 3, a = gl & 7;
-      const int32_t row0 = b * p.L_max;
+      const int32_t row0 = p.cm.paged() ? 0 : b * p.L_max;  // stand-in row for invalid keys
       auto load_rows = [&](int tile, int (&y)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -583,7 +584,10 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           if (active) {
             int y[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) y[i] = row0 + ((cur[i] >= 0 && cur[i] < len) ? cur[i] : 0);
+            for (int i = 0; i < 4; ++i) {
+              bool rok;
+              y[i] = (cur[i] >= 0 && cur[i] < len) ? p.cm.row(b, cur[i], rok) : row0;
+            }
             tma_gather4(smem_u32(smem + C::B_OFF_V + sl * C::V_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0],
                         y[1], y[2], y[3], &v_full[sl]);
           }

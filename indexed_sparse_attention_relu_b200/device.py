@@ -90,3 +90,40 @@ def subset(dw: DeviceWorkload, rows) -> DeviceWorkload:
     batch = B.Batch(torch.from_numpy(cu).to(dev), dw.batch.q_pos[r].contiguous(), dw.batch.seq_lens, wl.Lmax)
     return dataclasses.replace(dw, wl=sub_wl, batch=batch, q_idx=dw.q_idx[r].contiguous(), w=dw.w[r].contiguous(),
                                q=dw.q[r].contiguous())
+
+
+def to_paged(dw: DeviceWorkload, page_size: int, seed: int = 0, spare_pages: int = 3,
+             fill: float = 1000.0) -> DeviceWorkload:
+    """The same workload with every cache moved into one page pool.
+
+    Page placement comes from :func:`.workloads.page_layout`; rows are copied
+    page by page (layout only). Pool rows no sequence owns hold ``fill`` (FP8
+    codes: 0x7E, scales: 1), so a kernel that read a wrong row would show it.
+    """
+    from . import workloads as W
+    wl = dw.wl
+    table, num_pages = W.page_layout(wl.seq_lens, wl.Lmax, page_size, seed, spare_pages)
+    rows = num_pages * page_size
+    src = np.full(rows, -1, np.int64)
+    for b in range(wl.B):
+        for j in np.nonzero(table[b] >= 0)[0]:
+            n = min(page_size, wl.Lmax - int(j) * page_size)
+            pg = int(table[b, j])
+            src[pg * page_size:pg * page_size + n] = b * wl.Lmax + int(j) * page_size + np.arange(n)
+    dev = dw.q.device
+    src_t = torch.from_numpy(src).to(dev)
+    have = src_t >= 0
+
+    def scatter(cache: torch.Tensor, fill_value) -> torch.Tensor:
+        flat = cache.reshape(wl.B * wl.Lmax, -1)
+        pool = torch.full((rows, flat.shape[1]), fill_value, dtype=cache.dtype, device=dev)
+        pool[have] = flat[src_t[have]]
+        return pool
+
+    fp8 = dw.k_scale is not None
+    k_cache = scatter(dw.k_cache, 0x7E if fp8 else fill)
+    k_scale = scatter(dw.k_scale, 1.0) if fp8 else None
+    kv = scatter(dw.kv, fill)
+    batch = B.Batch(dw.batch.cu_q, dw.batch.q_pos, dw.batch.seq_lens, wl.Lmax,
+                    block_table=torch.from_numpy(table).to(dev), page_size=page_size, num_pages=num_pages)
+    return dataclasses.replace(dw, batch=batch, k_cache=k_cache, k_scale=k_scale, kv=kv, k_bf16=None)

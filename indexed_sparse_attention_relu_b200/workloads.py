@@ -366,3 +366,24 @@ def restrict(wl: Workload, rows) -> Workload:
 
 
 CONFIGS = tuple(_SEEDS)
+
+
+def page_layout(seq_lens, Lmax: int, page_size: int, seed: int, spare_pages: int = 3):
+    """A seeded random placement of every sequence's cache pages in one pool.
+
+    Sequence b needs ceil(seq_lens[b] / page_size) pages; they get distinct
+    pool pages drawn in random order from a pool with ``spare_pages`` pages
+    nobody uses. Returns (block_table [B, ceil(Lmax / page_size)] int32, with
+    -1 in every entry a sequence does not need, num_pages).
+    """
+    lens = np.asarray(seq_lens, np.int64)
+    max_pages = (Lmax + page_size - 1) // page_size
+    need = (lens + page_size - 1) // page_size
+    num_pages = int(need.sum()) + spare_pages
+    order = np.random.Generator(np.random.Philox(key=_key(seed, "pages"))).permutation(num_pages)
+    table = np.full((len(lens), max_pages), -1, np.int32)
+    pos = 0
+    for b, n in enumerate(need):
+        table[b, :n] = order[pos:pos + n]
+        pos += int(n)
+    return table, num_pages

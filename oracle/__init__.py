@@ -185,3 +185,23 @@ def dsa(wl, rows=None, *, k_codes=None, k_scales=None, rank_in_fp32: bool = Fals
     idx = topk(rank, nv, wl.K)
     out, lse = sparse_mla(wl, idx, rows)
     return sc, idx, out, lse
+
+
+def unpage(pool: np.ndarray, block_table: np.ndarray, page_size: int, Lmax: int) -> np.ndarray:
+    """The logical cache [B, Lmax, ...] of a page pool [num_pages * page_size, ...].
+
+    Paged caches (the fused indexer reads the paged key cache directly:
+    section 3 of "Optimizing Inference for New Model Architectures ..."):
+    row s of sequence b is pool row
+        block_table[b, s // page_size] * page_size + s % page_size.
+    Rows of a page whose table entry is -1 are zero. Plain loops over rows
+    (small cases only)."""
+    pool = np.asarray(pool)
+    table = np.asarray(block_table)
+    out = np.zeros((table.shape[0], Lmax) + pool.shape[1:], pool.dtype)
+    for b in range(table.shape[0]):
+        for s in range(Lmax):
+            pg = int(table[b, s // page_size])
+            if pg >= 0:
+                out[b, s] = pool[pg * page_size + s % page_size]
+    return out

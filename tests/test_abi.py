@@ -73,7 +73,17 @@ def test_indexer_validation(lib):
     assert lib.dsa_indexer_scores(None, ctypes.byref(_idx_in()), FAKE, 256, None, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
     assert _scores(lib, _batch(batch=0), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
     assert _scores(lib, _batch(cu_q=None), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
+    # paged caches: page_size a positive multiple of 64, a positive page count,
+    # a pool below 2^31 rows, an aligned table; no paging fields without a table
     assert _scores(lib, _batch(block_table=FAKE), _idx_in()) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(block_table=FAKE, page_size=96, num_pages=4), _idx_in()) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(block_table=FAKE, page_size=64, num_pages=0), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(block_table=FAKE, page_size=1 << 16, num_pages=1 << 15), _idx_in()) == \
+        B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(block_table=FAKE + 2, page_size=64, num_pages=8), _idx_in()) == B.DSA_ERR_MISALIGNED
+    assert _scores(lib, _batch(page_size=64), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(num_pages=3), _idx_in()) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(block_table=FAKE, page_size=128, num_pages=8, num_q=0), _idx_in()) == B.DSA_OK
     assert _scores(lib, _batch(), _idx_in(n_heads=32)) == B.DSA_ERR_UNSUPPORTED_SHAPE
     assert _scores(lib, _batch(), _idx_in(head_dim=96)) == B.DSA_ERR_UNSUPPORTED_SHAPE
     assert _scores(lib, _batch(), _idx_in(q=MIS)) == B.DSA_ERR_MISALIGNED

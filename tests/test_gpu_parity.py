@@ -93,6 +93,47 @@ def test_indexer_fp8_ragged_decode():
 
 
 @pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
+@pytest.mark.parametrize("HI,dI", [(4, 32), (4, 128), (64, 32), (64, 128)])
+def test_indexer_decode_shapes_integer_exact(HI, dI, key_dtype):
+    """One query per sequence (the balanced decode kernel) for every supported
+    indexer shape, integer values in [-2, 2] so every score is exact: BF16 keys
+    give integer sums, FP8 keys give codes in {0, +-224, +-448} times one scale
+    applied after the head sum (fl32 of an exact value)."""
+    wl = W.scaled("c5i", B=5, Lmax=700, lens=(700, 129, 128, 1, 513), T_per_seq=1, K=64, HI=HI, dI=dI,
+                  key_dtype=key_dtype, integer=True)
+    dw = DV.to_device(wl)
+    kw = {}
+    if key_dtype == "fp8":
+        codes, scales = oracle_codes(dw)
+        kw = dict(k_codes=codes, k_scales=scales)
+    got = _np(gpu_scores(dw))
+    want = oracle.indexer_scores(wl, **kw)
+    nv = wl.n_valid()
+    for t in range(wl.T):
+        assert np.array_equal(got[t, :nv[t]], want[t, :nv[t]].astype(np.float32)), t
+        assert np.all(got[t, nv[t]:(nv[t] + 127) // 128 * 128] == -np.inf)
+
+
+@pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
+def test_indexer_decode_ranges_span_many_tokens(key_dtype):
+    """200 short sequences (one of them empty): the flattened key-tile list has
+    fewer tiles than twice the CTA count, so CTA ranges start and end inside
+    tokens and run across several of them."""
+    rng = np.random.default_rng(21)
+    lens = rng.integers(1, 400, 200)
+    lens[17] = 0
+    wl = W.scaled("c2", B=200, Lmax=400, lens=tuple(int(x) for x in lens), T_per_seq=1, K=128, key_dtype=key_dtype)
+    dw = DV.to_device(wl)
+    kw = {}
+    if key_dtype == "fp8":
+        codes, scales = oracle_codes(dw)
+        kw = dict(k_codes=codes, k_scales=scales)
+    got = _np(gpu_scores(dw))
+    want = oracle.indexer_scores(wl, **kw)
+    check_scores(got, want, score_bound(wl, **kw), wl.n_valid())
+
+
+@pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
 def test_indexer_causal_prefill_groups(key_dtype):
     """Several tokens per sequence: the 4-token MMA groups, causal masks that
     differ inside a group, and groups that end mid-sequence."""
