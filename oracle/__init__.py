@@ -60,7 +60,7 @@ def _load():
             lib.oracle_topk.argtypes = [ctypes.c_int32, _f64p, ctypes.c_int64, _i32p, ctypes.c_int32, _i32p]
             lib.oracle_sparse_mla.argtypes = [
                 ctypes.c_int32, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
-                ctypes.c_double, _f32p, _f32p, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32, _f64p, _f64p]
+                ctypes.c_double, _f32p, _f64p, ctypes.c_int32, _i32p, _i32p, ctypes.c_int32, _f64p, _f64p]
             lib.oracle_num_threads.restype = ctypes.c_int32
             lib.oracle_set_num_threads.argtypes = [ctypes.c_int32]
             _lib = lib
@@ -156,8 +156,11 @@ def topk(scores: np.ndarray, n_valid, K: int) -> np.ndarray:
     return out
 
 
-def sparse_mla(wl, idx: np.ndarray, rows=None):
-    """Attention over the selected rows: returns (out [n,H,dc] fp64, lse [n,H] fp64)."""
+def sparse_mla(wl, idx: np.ndarray, rows=None, kv=None):
+    """Attention over the selected rows: returns (out [n,H,dc] fp64, lse [n,H] fp64).
+
+    ``kv`` replaces the workload's bf16 latent rows (e.g. the FP8 cache's
+    rows dequantised in fp64 by :func:`dequantize_kv`)."""
     lib = _load()
     rows = np.arange(wl.T, dtype=np.int32) if rows is None else _c(rows, np.int32)
     idx = _c(idx, np.int32)
@@ -165,9 +168,10 @@ def sparse_mla(wl, idx: np.ndarray, rows=None):
     out = np.empty((len(rows), wl.H, wl.dc), np.float64)
     lse = np.empty((len(rows), wl.H), np.float64)
     cu_q, lens = _c(wl.cu_q, np.int32), _c(wl.seq_lens, np.int32)
-    q, kv = _c(wl.q, np.float32), _c(wl.kv, np.float32)
+    q = _c(wl.q, np.float32)
+    kv = _c(wl.kv if kv is None else kv, np.float64)
     lib.oracle_sparse_mla(wl.B, wl.Lmax, _p(cu_q, _i32p), _p(lens, _i32p), wl.H, wl.D, wl.dc,
-                          float(wl.softmax_scale), _p(q, _f32p), _p(kv, _f32p), len(rows),
+                          float(wl.softmax_scale), _p(q, _f32p), _p(kv, _f64p), len(rows),
                           _p(rows, _i32p), _p(idx, _i32p), K, _p(out, _f64p), _p(lse, _f64p))
     return out, lse
 
@@ -205,3 +209,26 @@ def unpage(pool: np.ndarray, block_table: np.ndarray, page_size: int, Lmax: int)
             if pg >= 0:
                 out[b, s] = pool[pg * page_size + s % page_size]
     return out
+
+
+def quantize_kv(kv: np.ndarray, dc: int, tile: int = 128):
+    """FP8 cache write of latent KV rows [..., dc + d_rope] (Block-Wise
+    Quantization for Key-Value Cache: "Optimizing Inference for New Model
+    Architectures ...", section 4; Tiered Quantization table of "Day-0
+    Inference Adaptation ..."): the dc latent dims in tiles of ``tile``
+    elements (one tile when dc < tile), each with scale = absmax / 448 and
+    codes e4m3(round to nearest even, saturating)(x / scale) -- the same
+    per-group dynamic quantisation as the index keys; the rope dims stay bf16.
+    Returns (codes [..., dc] uint8, scales [..., dc / g] fp32, rope [..., d_rope] fp32)."""
+    kv = _c(kv, np.float32)
+    g = min(tile, dc)
+    codes, scales = quantize_keys(np.ascontiguousarray(kv[..., :dc]), g)
+    return codes, scales, np.ascontiguousarray(kv[..., dc:])
+
+
+def dequantize_kv(codes: np.ndarray, scales: np.ndarray, rope: np.ndarray) -> np.ndarray:
+    """fp64 latent rows of an FP8 KV cache: decode(code) * tile scale (exact in
+    fp64: a code carries 4 significant bits, a scale 24), then the rope dims."""
+    g = codes.shape[-1] // scales.shape[-1]
+    lat = e4m3_decode(codes) * np.repeat(np.asarray(scales, np.float64), g, axis=-1)
+    return np.concatenate([lat, np.asarray(rope, np.float64)], axis=-1)

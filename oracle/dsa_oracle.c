@@ -258,11 +258,12 @@ void oracle_topk(int32_t n_rows, const double *scores, int64_t ld, const int32_t
  *   out[r,h,:] = sum_i p_i * kv[b, s_i, 0:dc]        (value = latent part)
  *   lse[r,h] = m + log(sum_i exp(z_i - m))
  * No selected row: out = 0, lse = -inf.
- * q [T,H,D], kv [B,Lmax,D] (bf16-exact fp32), idx [n_rows, K];
+ * q [T,H,D] (bf16-exact fp32), kv [B,Lmax,D] fp64 (bf16 values, or FP8
+ * codes times their tile scale, exact in fp64), idx [n_rows, K];
  * out [n_rows, H, dc], lse [n_rows, H] (fp64). */
 void oracle_sparse_mla(int32_t B, int32_t Lmax, const int32_t *cu_q, const int32_t *seq_lens,
                        int32_t H, int32_t D, int32_t dc, double scale, const float *q,
-                       const float *kv, int32_t n_rows, const int32_t *rows, const int32_t *idx,
+                       const double *kv, int32_t n_rows, const int32_t *rows, const int32_t *idx,
                        int32_t K, double *out, double *lse)
 {
 #pragma omp parallel for collapse(2) schedule(dynamic, 4)
@@ -280,10 +281,10 @@ void oracle_sparse_mla(int32_t B, int32_t Lmax, const int32_t *cu_q, const int32
                 int32_t s = sel[i];
                 if (s < 0 || s >= seq_lens[b])
                     continue;
-                const float *kr = kv + ((int64_t)b * Lmax + s) * D;
+                const double *kr = kv + ((int64_t)b * Lmax + s) * D;
                 double dot = 0.0;
                 for (int32_t d = 0; d < D; ++d)
-                    dot += (double)qh[d] * (double)kr[d];
+                    dot += (double)qh[d] * kr[d];
                 z[n] = scale * dot;
                 rowid[n] = s;
                 ++n;
@@ -302,9 +303,9 @@ void oracle_sparse_mla(int32_t B, int32_t Lmax, const int32_t *cu_q, const int32
                     l += exp(z[i] - m);
                 for (int32_t i = 0; i < n; ++i) {
                     double p = exp(z[i] - m) / l;
-                    const float *vr = kv + ((int64_t)b * Lmax + rowid[i]) * D;
+                    const double *vr = kv + ((int64_t)b * Lmax + rowid[i]) * D;
                     for (int32_t d = 0; d < dc; ++d)
-                        o[d] += p * (double)vr[d];
+                        o[d] += p * vr[d];
                 }
                 lse[(int64_t)r * H + h] = m + log(l);
             }
