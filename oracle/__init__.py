@@ -232,3 +232,43 @@ def dequantize_kv(codes: np.ndarray, scales: np.ndarray, rope: np.ndarray) -> np
     g = codes.shape[-1] // scales.shape[-1]
     lat = e4m3_decode(codes) * np.repeat(np.asarray(scales, np.float64), g, axis=-1)
     return np.concatenate([lat, np.asarray(rope, np.float64)], axis=-1)
+
+
+def mx_quantize(x: np.ndarray, group: int = 32):
+    """MXFP8 per-group dynamic quantisation of index queries / keys [..., dim]
+    (Index Q/K Uses MXFP8, section 4.2 of "Inference Adaptation and
+    Performance Optimization for New Large Language Model Architectures";
+    every 32 elements share one scale factor).
+
+    Reading: the group's scale is the per-group pseudocode's absmax / 448
+    rounded up to a power of two 2^e -- the E8M0 shared scale of the MX
+    format, chosen so that no element saturates: e is the least integer
+    with 448 * 2^e >= absmax (an exact comparison), kept in [-127, 127];
+    absmax = 0 gives e = -127 and codes 0. Each element's code is the E4M3
+    cast (nearest even, saturating) of x / 2^e, which is exact before the
+    cast. Returns (codes uint8 [..., dim], scale bytes uint8 [..., dim / group]
+    holding e + 127)."""
+    x = np.asarray(x, np.float32)
+    dim = x.shape[-1]
+    g = x.reshape(-1, dim // group, group).astype(np.float64)
+    amax = np.abs(g).max(axis=-1)
+    e = np.full(amax.shape, -127, np.int64)
+    nz = amax > 0
+    e[nz] = np.floor(np.log2(amax[nz] / 448.0)).astype(np.int64) - 1
+    for _ in range(4):  # settle on the least e with 448 * 2^e >= absmax (exact in fp64)
+        up = nz & (448.0 * np.ldexp(1.0, e) < amax)
+        e[up] += 1
+    down = nz & (448.0 * np.ldexp(1.0, e - 1) >= amax)
+    assert not down.any()
+    e = np.clip(e, -127, 127)
+    scaled = (g * np.ldexp(1.0, -e)[..., None]).astype(np.float32)
+    codes = e4m3_encode(scaled).reshape(x.shape)
+    return codes, (e + 127).astype(np.uint8).reshape(x.shape[:-1] + (dim // group,))
+
+
+def mx_dequantize(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
+    """decode(code) * 2^(byte - 127), exact (fp64; also exact in fp32 and
+    bf16 while the result stays inside their normal range)."""
+    g = codes.shape[-1] // scale_bytes.shape[-1]
+    e = np.repeat(np.asarray(scale_bytes, np.int64) - 127, g, axis=-1)
+    return e4m3_decode(codes) * np.ldexp(1.0, e)
