@@ -5,12 +5,13 @@ Default workload: decode, batch 32 x 8192 context, one new token each
 (H_I=64, d_I=128, K=2048, 128 MLA heads, 512+64 latent dims, BF16), timed as
 one ``dsa_fused_decode`` call per step through the C ABI. Prints one JSON line.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c3|c4|c5] [--extra c3,c4,c5]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c3|c4|c5] [--extra c3,c3mx,c2kv8,c4,c5]
   python bench.py --impl reference ...     # the CPU oracle, timed on host cores
 
 The JSON line's headline is the decode workload; ``configs`` adds one block
-per extra workload (the ragged FP8-key decode against the HBM roofline, the
-prefills against the dense tensor-core peak), each graph-timed the same way.
+per extra workload (the ragged decode with FP8 or MXFP8 index inputs and the
+decode over an FP8 latent KV cache against the HBM roofline, the prefills
+against the dense tensor-core peak), each graph-timed the same way.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronize, timed with CUDA events on the launch stream; max over
@@ -45,7 +46,17 @@ WORKLOAD_TEXT = {
           "128 MLA heads, 576-dim BF16 latent rows",
     "c4": "causal prefill: 1 x 32768 tokens; H_I=64 d_I=128 BF16; K=2048; 128 MLA heads, 576/512 dims",
     "c5": "chunked prefill: 4 x (131072 prefix + 8192 chunk); FP8 index keys; K=2048; 128 MLA heads",
+    "c3mx": "ragged decode: batch 64, context U[1024,65536]; MXFP8 index queries and keys (E4M3, one E8M0 "
+            "scale per 32 elements); K=2048; 128 MLA heads, 576-dim BF16 latent rows",
+    "c2kv8": "decode: batch 32 x 8192 context, 1 query each; H_I=64 d_I=128 BF16 index keys; K=2048; "
+             "128 MLA heads; FP8 latent KV cache (4 x 128-element tiles per token, fp32 scales, rope BF16: "
+             "656-byte rows)",
 }
+
+# Workloads that are another one's inputs with the latent KV cache in FP8, or
+# with MXFP8 index queries and keys.
+FP8_KV = {"c2kv8": "c2"}
+MX_INDEX = {"c3mx": "c3"}
 
 
 def _peaks():
@@ -79,21 +90,24 @@ def algorithmic_flops(wl, n_selected: int):
     return {"indexer": idx, "sparse_mla": attn, "step": idx + attn}
 
 
-def algorithmic_bytes(wl, n_selected: int):
+def algorithmic_bytes(wl, n_selected: int, kv_row_bytes: int | None = None, key_row_bytes: int | None = None):
     """Bytes each stage must move at least once (inputs read + outputs written).
 
     indexer: index-key rows of every causal candidate, q_I, w, the fp32 score row
     written and read back by the Top-K; attention: the selected latent rows
-    (D bf16 each), q, idx and the bf16 output."""
+    (D bf16 each, or kv_row_bytes for an FP8 cache), q, idx and the bf16 output."""
     nv = wl.n_valid().astype(np.int64)
     key_row = wl.dI * (1 if wl.key_dtype == "fp8" else 2) + (4 if wl.key_dtype == "fp8" else 0)
+    if key_row_bytes is not None:  # MXFP8: codes + one scale byte per 32
+        key_row = key_row_bytes
     # distinct key rows read: every sequence's rows up to its longest causal history
     b = wl.seq_of_token()
     rows_per_seq = np.zeros(wl.B, np.int64)
     np.maximum.at(rows_per_seq, b, nv)
     idx_bytes = int(rows_per_seq.sum()) * key_row + wl.T * wl.HI * wl.dI * 2 + wl.T * wl.HI * 4
     scores = int(nv.sum()) * 4
-    attn = n_selected * wl.D * 2 + wl.T * wl.H * wl.D * 2 + wl.T * wl.K * 4 + wl.T * wl.H * wl.dc * 2
+    row = wl.D * 2 if kv_row_bytes is None else kv_row_bytes
+    attn = n_selected * row + wl.T * wl.H * wl.D * 2 + wl.T * wl.K * 4 + wl.T * wl.H * wl.dc * 2
     return {"indexer": idx_bytes + scores, "topk": scores + wl.T * wl.K * 4, "sparse_mla": attn,
             "step": idx_bytes + attn}
 
@@ -240,24 +254,34 @@ class Runner:
         from indexed_sparse_attention_relu_b200 import device as DV
         from indexed_sparse_attention_relu_b200 import workloads as W
         self.B = B
-        self.wl = wl = W.make(name, with_caches=False)
+        self.wl = wl = W.make(FP8_KV.get(name, MX_INDEX.get(name, name)), with_caches=False)
         self.dev = dev
-        base = DV.to_device(wl, dev)
+        base = DV.to_device(wl, dev, keep_bf16_keys=name in MX_INDEX)
+        self.kv_row_bytes = None
+        self.key_row_bytes = None
+        if name in MX_INDEX:  # the library's MXFP8 quantisation of q_I and k_I, outside the timed region
+            base = DV.with_mxfp8_index(base)
+            self.key_row_bytes = wl.dI + wl.dI // 32
+        if name in FP8_KV:  # the library's FP8 KV cache write, outside the timed region
+            base = DV.with_fp8_kv(base)
+            self.kv_row_bytes = B.dsa_kv_fp8_row_bytes(wl.dc, wl.dr)
         self.copies = [base]
         for _ in range(copies - 1):
             self.copies.append(DV.DeviceWorkload(wl, base.batch, base.q_idx.clone(), base.w.clone(),
                                                  base.k_cache.clone(),
                                                  None if base.k_scale is None else base.k_scale.clone(), None,
-                                                 base.q.clone(), base.kv.clone()))
+                                                 base.q.clone(), base.kv.clone(),
+                                                 None if base.q_mx is None else base.q_mx.clone(),
+                                                 None if base.k_mx is None else base.k_mx.clone()))
         T, K = wl.T, wl.K
         self.outs = [torch.empty((T, wl.H, wl.dc), dtype=torch.bfloat16, device=dev) for _ in self.copies]
         self.lses = [torch.empty((T, wl.H), dtype=torch.float32, device=dev) for _ in self.copies]
-        self.ws_bytes = B.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, base.batch, K)
+        self.ws_bytes = B.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, base.batch, K, wl.HI, wl.dI)
         self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
         self.idx_in = [c.indexer_in() for c in self.copies]
         self.mla_in = [c.mla_in() for c in self.copies]
-        self.resident_bytes = sum(c.kv.numel() * 2 + c.k_cache.numel() * c.k_cache.element_size() + c.q.numel() * 2
-                                  for c in self.copies)
+        self.resident_bytes = sum(c.kv.numel() * c.kv.element_size() + c.k_cache.numel() * c.k_cache.element_size()
+                                  + c.q.numel() * 2 for c in self.copies)
 
     def step(self, i, stream, events=None):
         j = i % len(self.copies)
@@ -390,7 +414,8 @@ def extra_block(name, args, dev, stream):
     """One graph-timed measurement of another workload, with its roofline."""
     import torch
     t0 = time.time()
-    steps = args.extra_steps_decode if name == "c3" else args.extra_steps_prefill
+    decode = name in ("c3", "c3mx", "c2kv8")
+    steps = args.extra_steps_decode if decode else args.extra_steps_prefill
     run = Runner(name, dev, copies=2)
     wl = run.wl
     total_ms, clocks, mode, status = time_steps(run, steps, 2, stream, dev)
@@ -401,12 +426,15 @@ def extra_block(name, args, dev, stream):
              "query_tokens_per_s": wl.T / (ms * 1e-3), "stage_ms": stages, "clocks": clocks, "timing": mode,
              "device_status": [status, run.B.dsa_read_device_status(stream)],
              "l2": f"2 rotating input copies ({run.resident_bytes / 1e9:.2f} GB) > 126 MB L2"}
-    if name == "c3":
+    if decode:
         peak, kind = _peaks()
-        b = algorithmic_bytes(wl, n_sel)["step"]
+        ab = algorithmic_bytes(wl, n_sel, run.kv_row_bytes, run.key_row_bytes)
+        b = ab["step"]
         block["roofline"] = {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
                              "frac": b / (ms * 1e-3) / 1e9 / peak, "peak_kind": kind, "algorithmic_bytes": b,
-                             "frac_of_8TBps": b / (ms * 1e-3) / 1e9 / 8000.0}
+                             "frac_of_8TBps": b / (ms * 1e-3) / 1e9 / 8000.0,
+                             "stage_frac": {k: ab[k] / (stages[k] * 1e-3) / 1e9 / peak
+                                            for k in ("indexer", "topk", "sparse_mla")}}
     else:
         burst, sustained, kind = _peak_tflops()
         f = algorithmic_flops(wl, n_sel)
@@ -435,7 +463,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=1, help="query tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph")
-    ap.add_argument("--extra", default="c3,c4,c5",
+    ap.add_argument("--extra", default="c3,c3mx,c2kv8,c4,c5",
                     help="comma-separated extra workloads measured after the headline (single GPU only; '' for none)")
     ap.add_argument("--extra-steps-decode", type=int, default=20)
     ap.add_argument("--extra-steps-prefill", type=int, default=3)

@@ -75,7 +75,15 @@ typedef enum {
                                        or an SM id outside its per-SM workspace records */
 } dsa_status;
 
-typedef enum { DSA_KEY_BF16 = 0, DSA_KEY_FP8_E4M3 = 1 } dsa_key_dtype;
+/* Index query / key formats:
+ *   DSA_KEY_BF16      bf16 queries and keys;
+ *   DSA_KEY_FP8_E4M3  bf16 queries, E4M3 key codes with one fp32 scale per key;
+ *   DSA_KEY_MXFP8     E4M3 codes for queries AND keys, one E8M0 (power-of-two)
+ *                     scale per 32 elements of each (Index Q/K Uses MXFP8,
+ *                     section 4.2 of "Inference Adaptation and Performance
+ *                     Optimization for New Large Language Model
+ *                     Architectures"); see dsa_quantize_mxfp8. */
+typedef enum { DSA_KEY_BF16 = 0, DSA_KEY_FP8_E4M3 = 1, DSA_KEY_MXFP8 = 2 } dsa_key_dtype;
 
 /* Ops for dsa_workspace_size(). */
 typedef enum {
@@ -125,13 +133,18 @@ typedef struct {
 } dsa_batch;
 
 /* Lightning Indexer inputs.
- *   q        bf16 [T, n_heads, head_dim]       indexer queries q_I
+ *   q        [T, n_heads, head_dim]            indexer queries q_I: bf16, or
+ *            E4M3 codes (DSA_KEY_MXFP8)
  *   w        fp32 [T, n_heads]                 head weights
  *   k_cache  [rows, head_dim]                  index keys, bf16 or e4m3 codes;
  *            rows = B * L_max (contiguous) or num_pages * page_size (paged)
- *   k_scale  fp32 [rows, head_dim/scale_group] per-group scales (FP8 only;
- *            the key value is decode(code) * scale), NULL for BF16
- *   scale_group: elements per scale; must equal head_dim for the FP8 indexer. */
+ *   k_scale  fp32 [rows, head_dim/scale_group] per-group scales (FP8_E4M3
+ *            only; the key value is decode(code) * scale), else NULL
+ *   scale_group: elements per scale; head_dim for FP8_E4M3 (one scale per
+ *            key), 32 for MXFP8.
+ *   q_scale_e8m0  uint8 [T, n_heads, head_dim/32], k_scale_e8m0 uint8
+ *            [rows, head_dim/32]: MXFP8 scale bytes (value = decode(code) *
+ *            2^(byte - 127)), else NULL. */
 typedef struct {
     int32_t n_heads;
     int32_t head_dim;
@@ -141,13 +154,25 @@ typedef struct {
     const void *k_cache;
     const float *k_scale;
     int32_t scale_group;
+    const uint8_t *q_scale_e8m0;
+    const uint8_t *k_scale_e8m0;
 } dsa_indexer_in;
+
+/* Latent KV cache element types. */
+typedef enum { DSA_KV_BF16 = 0, DSA_KV_FP8_E4M3 = 1 } dsa_kv_dtype;
 
 /* Sparse MLA inputs.
  *   q   bf16 [T, n_heads, d_latent + d_rope]
- *   kv  bf16 [rows, d_latent + d_rope]   latent rows (rows as for k_cache);
- *       value = first d_latent
- *   softmax_scale: multiplies q . kv before the softmax. */
+ *   kv  latent rows (rows as for k_cache); value = first d_latent dims:
+ *       DSA_KV_BF16:     bf16 [rows, d_latent + d_rope]
+ *       DSA_KV_FP8_E4M3: packed FP8 rows [rows, dsa_kv_fp8_row_bytes()] as
+ *                        written by dsa_quantize_kv (block-wise FP8 KV cache:
+ *                        section 4 of "Optimizing Inference for New Model
+ *                        Architectures ..."). The rows are widened to bf16
+ *                        on chip (fl32(decode(code) * tile scale) rounded to
+ *                        nearest bf16); q and the products stay bf16/fp32.
+ *   softmax_scale: multiplies q . kv before the softmax.
+ *   kv_dtype: DSA_KV_BF16 (0) or DSA_KV_FP8_E4M3. */
 typedef struct {
     int32_t n_heads;
     int32_t d_latent;
@@ -155,6 +180,7 @@ typedef struct {
     float softmax_scale;
     const void *q;
     const void *kv;
+    dsa_kv_dtype kv_dtype;
 } dsa_mla_in;
 
 /* Lightning Indexer scores (relevance scoring + head-weight weighting +
@@ -164,8 +190,12 @@ typedef struct {
  *   last 128-key tile that holds a valid key; entries beyond are not written.
  * FP8 keys: I = scale_s * sum_j w_j * max(0, q_j . decode(code_s)), which
  * equals the score of the dequantised key because scale_s >= 0.
- * ws: workspace of dsa_workspace_size(DSA_OP_INDEXER_SCORES, ...) bytes (may
- * be NULL when that size is 0). */
+ * MXFP8: the scores of the dequantised queries and keys; every dequantised
+ * element is exact in bf16, so the products are exact and only the fp32
+ * sums round, as for bf16 inputs.
+ * ws: workspace of dsa_workspace_size(DSA_OP_INDEXER_SCORES, ...) bytes,
+ * 16-byte aligned; used only by MXFP8 (the widened queries: T * n_heads *
+ * head_dim * 2 bytes), may be NULL otherwise. */
 dsa_status dsa_indexer_scores(const dsa_batch *batch, const dsa_indexer_in *in, float *scores,
                               int64_t score_ld, void *ws, size_t ws_bytes, dsa_stream_t stream);
 
@@ -234,7 +264,9 @@ dsa_status dsa_fused_decode(const dsa_batch *batch, const dsa_indexer_in *idx_in
  * capture.
  * All calls share the array: calls whose work overlaps on the GPU (other
  * streams, other threads) race on it and must be serialised by the caller.
- * Nothing in the array needs to start at zero; stale contents are never read. */
+ * Nothing in the array needs to start at zero; stale contents are never read.
+ * MXFP8 index inputs are not accepted here (DSA_ERR_UNSUPPORTED_SHAPE): their
+ * widened queries would need more scratch. */
 dsa_status dsa_fused_decode_noalloc(const dsa_batch *batch, const dsa_indexer_in *idx_in,
                                     const dsa_mla_in *mla_in, int32_t k, void *out, float *lse,
                                     int32_t *idx_out, dsa_stream_t stream);
@@ -253,15 +285,49 @@ dsa_status dsa_fused_decode_noalloc(const dsa_batch *batch, const dsa_indexer_in
 dsa_status dsa_quantize_index_keys(const void *k_bf16, int64_t n_keys, int32_t dim, int32_t group,
                                    uint8_t *k8, float *scale, dsa_stream_t stream);
 
+/* Latent KV cache write, FP8 (Block-Wise Quantization for Key-Value Cache,
+ * section 4 of "Optimizing Inference for New Model Architectures ..."; the
+ * Tiered Quantization table of "Day-0 Inference Adaptation ..."): per token
+ * row of kv_bf16 [n_rows, d_latent + d_rope], the d_latent dims in tiles of
+ * min(128, d_latent) elements, each with scale = fl32(max|x| / 448) and codes
+ * as in dsa_quantize_index_keys; the d_rope dims are kept in bf16. One packed
+ * row of dsa_kv_fp8_row_bytes(d_latent, d_rope) bytes per token:
+ *   bytes [0, d_latent)                       E4M3 codes
+ *   bytes [d_latent, d_latent + 2 d_rope)     rope dims, bf16
+ *   then one fp32 scale per tile, then zeros up to a multiple of 16 bytes
+ *   ((512, 64): 656 bytes; (64, 16): 112 bytes).
+ * (d_latent, d_rope) in {(512, 64), (64, 16)}; both pointers 16-byte aligned.
+ * Writes kv_fp8 only. */
+dsa_status dsa_quantize_kv(const void *kv_bf16, int64_t n_rows, int32_t d_latent, int32_t d_rope,
+                           uint8_t *kv_fp8, dsa_stream_t stream);
+
+/* Bytes of one packed FP8 latent row (see dsa_quantize_kv); 0 for
+ * unsupported dims. */
+size_t dsa_kv_fp8_row_bytes(int32_t d_latent, int32_t d_rope);
+
+/* MXFP8 quantisation of index queries or keys (Index Q/K Uses MXFP8, section
+ * 4.2 of "Inference Adaptation and Performance Optimization for New Large
+ * Language Model Architectures"; 32 elements share one scale). For each
+ * group of 32 elements of x_bf16 [n_rows, dim]: e = the least integer with
+ * 448 * 2^e >= max|x| (the group pseudocode's max / 448 rounded up to a power
+ * of two, so nothing saturates), kept in [-127, 127] (-127 for an all-zero
+ * group); scales[group] = e + 127 (E8M0); codes = E4M3 round-to-nearest-even
+ * of x * 2^-e (an exact product). dim a multiple of 32, <= 1024; all
+ * pointers 16-byte aligned. Writes codes [n_rows, dim] and scales
+ * [n_rows, dim / 32]. */
+dsa_status dsa_quantize_mxfp8(const void *x_bf16, int64_t n_rows, int32_t dim, uint8_t *codes, uint8_t *scales,
+                              dsa_stream_t stream);
+
 /* Inverse of the cache write above (same passage): the value a key's FP8
  * code stands for, out = fl32(decode(code) * scale), fp32 [n_keys, dim].
  * Same group and dim rules as dsa_quantize_index_keys. */
 dsa_status dsa_dequantize_index_keys(const uint8_t *k8, const float *scale, int64_t n_keys,
                                      int32_t dim, int32_t group, float *out, dsa_stream_t stream);
 
-/* Workspace bytes `op` needs for this batch, k and indexer shape (h_i, d_i);
- * the MLA shape is fixed by the supported set, the largest is assumed.
- * Host-only: reads no device memory. */
+/* Workspace bytes `op` needs for this batch, k and indexer shape (h_i, d_i),
+ * enough for every index-key format (MXFP8 needs room for the widened
+ * queries); the MLA shape is fixed by the supported set, the largest is
+ * assumed. Host-only: reads no device memory. */
 size_t dsa_workspace_size(int op, const dsa_batch *batch, int32_t k, int32_t h_i, int32_t d_i);
 
 /* Waits for `stream`, then returns in *code_out the sticky device status

@@ -33,6 +33,9 @@ DSA_ERR_DEVICE_LAYOUT = 8
 
 DSA_KEY_BF16 = 0
 DSA_KEY_FP8_E4M3 = 1
+DSA_KEY_MXFP8 = 2
+DSA_KV_BF16 = 0
+DSA_KV_FP8_E4M3 = 1
 
 DSA_OP_INDEXER_SCORES = 0
 DSA_OP_TOPK = 1
@@ -42,7 +45,9 @@ DSA_OP_FUSED_DECODE = 3
 # Every symbol include/dsa.h declares.
 EXPORTED = (
     "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_fused_decode", "dsa_fused_decode_noalloc",
-    "dsa_quantize_index_keys", "dsa_dequantize_index_keys", "dsa_workspace_size",
+    "dsa_quantize_index_keys", "dsa_dequantize_index_keys", "dsa_quantize_kv", "dsa_kv_fp8_row_bytes",
+    "dsa_quantize_mxfp8",
+    "dsa_workspace_size",
     "dsa_read_device_status", "dsa_status_string", "dsa_last_error", "dsa_version",
     "dsa_debug_set_wait_limit", "dsa_debug_withhold_signal",
 )
@@ -62,12 +67,13 @@ class dsa_batch(ctypes.Structure):
 
 class dsa_indexer_in(ctypes.Structure):
     _fields_ = [("n_heads", c_int32), ("head_dim", c_int32), ("q", c_void_p), ("w", c_void_p),
-                ("key_dtype", c_int32), ("k_cache", c_void_p), ("k_scale", c_void_p), ("scale_group", c_int32)]
+                ("key_dtype", c_int32), ("k_cache", c_void_p), ("k_scale", c_void_p), ("scale_group", c_int32),
+                ("q_scale_e8m0", c_void_p), ("k_scale_e8m0", c_void_p)]
 
 
 class dsa_mla_in(ctypes.Structure):
     _fields_ = [("n_heads", c_int32), ("d_latent", c_int32), ("d_rope", c_int32), ("softmax_scale", c_float),
-                ("q", c_void_p), ("kv", c_void_p)]
+                ("q", c_void_p), ("kv", c_void_p), ("kv_dtype", c_int32)]
 
 
 _lib = None
@@ -92,6 +98,9 @@ def load() -> ctypes.CDLL:
                                                  c_int32, P, P, P, P]),
             "dsa_quantize_index_keys": (c_int, [P, c_int64, c_int32, c_int32, P, P, P]),
             "dsa_dequantize_index_keys": (c_int, [P, P, c_int64, c_int32, c_int32, P, P]),
+            "dsa_quantize_kv": (c_int, [P, c_int64, c_int32, c_int32, P, P]),
+            "dsa_quantize_mxfp8": (c_int, [P, c_int64, c_int32, P, P, P]),
+            "dsa_kv_fp8_row_bytes": (c_size_t, [c_int32, c_int32]),
             "dsa_workspace_size": (c_size_t, [c_int, POINTER(dsa_batch), c_int32, c_int32, c_int32]),
             "dsa_read_device_status": (c_int, [P, POINTER(c_int32)]),
             "dsa_status_string": (c_char_p, [c_int]),
@@ -156,16 +165,26 @@ class Batch:
 
 
 def indexer_in(q: torch.Tensor, w: torch.Tensor, k_cache: torch.Tensor, k_scale: torch.Tensor | None = None,
-               scale_group: int | None = None) -> dsa_indexer_in:
-    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
+               scale_group: int | None = None, q_mx: torch.Tensor | None = None,
+               k_mx: torch.Tensor | None = None) -> dsa_indexer_in:
+    """BF16 keys; FP8 keys (uint8 codes + fp32 ``k_scale``); or MXFP8 queries
+    and keys (uint8 codes for both, E8M0 bytes ``q_mx`` / ``k_mx``)."""
     T, HI, DI = q.shape
+    if q_mx is not None:
+        return dsa_indexer_in(HI, DI, _ptr(q), _ptr(w), DSA_KEY_MXFP8, _ptr(k_cache), None, 32, _ptr(q_mx),
+                              _ptr(k_mx))
+    fp8 = k_cache.dtype in (torch.uint8, torch.float8_e4m3fn)
     return dsa_indexer_in(HI, DI, _ptr(q), _ptr(w), DSA_KEY_FP8_E4M3 if fp8 else DSA_KEY_BF16, _ptr(k_cache),
-                          _ptr(k_scale), int(scale_group if scale_group is not None else DI))
+                          _ptr(k_scale), int(scale_group if scale_group is not None else DI), None, None)
 
 
 def mla_in(q: torch.Tensor, kv: torch.Tensor, d_latent: int, softmax_scale: float) -> dsa_mla_in:
+    """bf16 latent rows, or packed FP8 rows (a uint8 tensor written by
+    dsa_quantize_kv)."""
     T, H, D = q.shape
-    return dsa_mla_in(H, int(d_latent), int(D - d_latent), float(softmax_scale), _ptr(q), _ptr(kv))
+    fp8 = kv.dtype == torch.uint8
+    return dsa_mla_in(H, int(d_latent), int(D - d_latent), float(softmax_scale), _ptr(q), _ptr(kv),
+                      DSA_KV_FP8_E4M3 if fp8 else DSA_KV_BF16)
 
 
 # ----------------------------------------------------------------------------- C-ABI calls
@@ -224,6 +243,22 @@ def dsa_quantize_index_keys(k_bf16: torch.Tensor, group: int, k8: torch.Tensor, 
     dim = k_bf16.shape[-1]
     _check(load().dsa_quantize_index_keys(_ptr(k_bf16), k_bf16.numel() // dim, dim, group, _ptr(k8), _ptr(scale),
                                           _stream(stream)))
+
+
+def dsa_quantize_mxfp8(x_bf16: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    dim = x_bf16.shape[-1]
+    _check(load().dsa_quantize_mxfp8(_ptr(x_bf16), x_bf16.numel() // dim, dim, _ptr(codes), _ptr(scales),
+                                     _stream(stream)))
+
+
+def dsa_kv_fp8_row_bytes(d_latent: int, d_rope: int) -> int:
+    return int(load().dsa_kv_fp8_row_bytes(d_latent, d_rope))
+
+
+def dsa_quantize_kv(kv_bf16: torch.Tensor, d_latent: int, kv_fp8: torch.Tensor, stream=None) -> None:
+    D = kv_bf16.shape[-1]
+    _check(load().dsa_quantize_kv(_ptr(kv_bf16), kv_bf16.numel() // D, d_latent, D - d_latent, _ptr(kv_fp8),
+                                  _stream(stream)))
 
 
 def dsa_dequantize_index_keys(k8: torch.Tensor, scale: torch.Tensor, group: int, out: torch.Tensor,

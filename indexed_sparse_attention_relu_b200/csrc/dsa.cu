@@ -155,7 +155,7 @@ dsa_status check_indexer(const dsa_batch* bt, const dsa_indexer_in* in) {
   if (!shape_ok)
     return fail(DSA_ERR_UNSUPPORTED_SHAPE, "indexer heads/dim %d/%d not in {4,64} x {32,128}", in->n_heads,
                 in->head_dim);
-  if (in->key_dtype != DSA_KEY_BF16 && in->key_dtype != DSA_KEY_FP8_E4M3)
+  if (in->key_dtype != DSA_KEY_BF16 && in->key_dtype != DSA_KEY_FP8_E4M3 && in->key_dtype != DSA_KEY_MXFP8)
     return fail(DSA_ERR_INVALID_ARGUMENT, "bad key dtype %d", static_cast<int>(in->key_dtype));
   if (!in->q || !in->w || !in->k_cache) return fail(DSA_ERR_INVALID_ARGUMENT, "indexer q, w, k_cache must be non-NULL");
   if (!aligned16(in->q) || !aligned16(in->w) || !aligned16(in->k_cache))
@@ -164,6 +164,12 @@ dsa_status check_indexer(const dsa_batch* bt, const dsa_indexer_in* in) {
     if (!in->k_scale) return fail(DSA_ERR_INVALID_ARGUMENT, "FP8 keys need k_scale");
     if (in->scale_group != in->head_dim)
       return fail(DSA_ERR_UNSUPPORTED_SHAPE, "FP8 indexer needs one scale per key (scale_group == head_dim)");
+  }
+  if (in->key_dtype == DSA_KEY_MXFP8) {
+    if (!in->q_scale_e8m0 || !in->k_scale_e8m0)
+      return fail(DSA_ERR_INVALID_ARGUMENT, "MXFP8 needs q_scale_e8m0 and k_scale_e8m0");
+    if (in->scale_group != 32) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "MXFP8 needs scale_group == 32");
+    if (!aligned16(in->q_scale_e8m0)) return fail(DSA_ERR_MISALIGNED, "q_scale_e8m0 must be 16-byte aligned");
   }
   (void)bt;
   return DSA_OK;
@@ -179,6 +185,8 @@ dsa_status check_mla(const dsa_mla_in* in) {
   if (!in->q || !in->kv) return fail(DSA_ERR_INVALID_ARGUMENT, "MLA q and kv must be non-NULL");
   if (!aligned16(in->q) || !aligned16(in->kv)) return fail(DSA_ERR_MISALIGNED, "MLA q and kv must be 16-byte aligned");
   if (!std::isfinite(in->softmax_scale)) return fail(DSA_ERR_INVALID_ARGUMENT, "softmax_scale must be finite");
+  if (in->kv_dtype != DSA_KV_BF16 && in->kv_dtype != DSA_KV_FP8_E4M3)
+    return fail(DSA_ERR_INVALID_ARGUMENT, "bad kv dtype %d", static_cast<int>(in->kv_dtype));
   return DSA_OK;
 }
 
@@ -293,14 +301,27 @@ dsa_status set_smem(Kern k, int bytes) {
   return DSA_OK;
 }
 
-template <int HI, int DIN, int G, bool FP8>
+// Key format of a call (the kernels' KF template argument).
+int key_format(const dsa_indexer_in* in) {
+  return in->key_dtype == DSA_KEY_MXFP8 ? KF_MX : in->key_dtype == DSA_KEY_FP8_E4M3 ? KF_FP8 : KF_BF16;
+}
+
+// Scale rows of 8-bit keys start on 16-byte boundaries at every tile (128
+// rows, or 64 when paged) when the base is aligned and, for contiguous
+// caches, L_max times the row's scale bytes is a multiple of 16.
+bool scale_rows_aligned(const dsa_batch* bt, const void* base, int row_bytes) {
+  return base && aligned16(base) && (bt->block_table || (static_cast<int64_t>(bt->max_seq_len) * row_bytes) % 16 == 0);
+}
+
+template <int HI, int DIN, int G, int KF>
 dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
                             cudaStream_t st, bool pdl) {
-  using C = IndexerCfg<HI, DIN, G, FP8>;
+  using C = IndexerCfg<HI, DIN, G, KF>;
+  constexpr bool FP8 = C::FP8;
   CUtensorMap map;
   dsa_status s = make_key_map(&map, in->k_cache, cache_rows(bt), DIN, FP8, key_box_rows(bt));
   if (s != DSA_OK) return s;
-  auto kern = indexer_scores_kernel<HI, DIN, G, FP8>;
+  auto kern = indexer_scores_kernel<HI, DIN, G, KF>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
   const int sms = num_sms();
   const int64_t groups64 = static_cast<int64_t>((bt->num_q + G - 1) / G) + bt->batch;
@@ -330,7 +351,10 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   p.cm = cache_map(bt);
   p.q = static_cast<const __nv_bfloat16*>(in->q);
   p.w = in->w;
-  p.k_scale = in->k_scale;
+  p.k_scale = KF == KF_FP8 ? in->k_scale : nullptr;
+  p.k_mx = KF == KF_MX ? in->k_scale_e8m0 : nullptr;
+  p.scale_bulk = KF == KF_MX && scale_rows_aligned(bt, in->k_scale_e8m0, DIN / 32);
+  p.rows = cache_rows(bt);
   p.scores = scores;
   p.ld = ld;
   p.tiles_per_cta = tpc;
@@ -351,21 +375,28 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
 
 // One query token per group (decode): one CTA per SM, each taking an equal
 // range of the flattened key-tile list of all tokens.
-template <int HI, int DIN, bool FP8>
+template <int HI, int DIN, int KF>
 dsa_status launch_indexer_decode(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
                                  cudaStream_t st, bool pdl) {
-  using C = IdxDecCfg<HI, DIN, FP8>;
+  using C = IdxDecCfg<HI, DIN, KF>;
+  constexpr bool FP8 = C::FP8;
   CUtensorMap kmap, qmap;
   dsa_status s = make_key_map(&kmap, in->k_cache, cache_rows(bt), DIN, FP8, key_box_rows(bt));
   if (s != DSA_OK) return s;
   if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(bt->num_q) * HI, DIN, HI)) != DSA_OK) return s;
-  auto kern = indexer_decode_kernel<HI, DIN, FP8>;
+  auto kern = indexer_decode_kernel<HI, DIN, KF>;
   if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
   IdxDecParams p;
   p.cu_q = bt->cu_q;
   p.q_pos = bt->q_pos;
   p.seq_lens = bt->seq_lens;
-  p.k_scale = FP8 ? in->k_scale : nullptr;
+  p.k_scale = KF == KF_FP8 ? in->k_scale : nullptr;
+  p.k_mx = KF == KF_MX ? in->k_scale_e8m0 : nullptr;
+  // the scales ride in the key stage when every tile's scale rows start on a
+  // 16-byte boundary
+  p.scale_bulk = FP8 && scale_rows_aligned(bt, KF == KF_MX ? static_cast<const void*>(in->k_scale_e8m0)
+                                                           : static_cast<const void*>(in->k_scale), C::SROW);
+  p.rows = cache_rows(bt);
   p.B = bt->batch;
   p.T = bt->num_q;
   p.L_max = bt->max_seq_len;
@@ -390,24 +421,47 @@ dsa_status launch_indexer_decode(const dsa_batch* bt, const dsa_indexer_in* in, 
 template <int HI, int DIN>
 dsa_status launch_indexer_g(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
                             cudaStream_t st, bool pdl) {
-  const bool fp8 = in->key_dtype == DSA_KEY_FP8_E4M3;
+  const int kf = key_format(in);
   // decode (one token per group): the balanced one-CTA-per-SM kernel while a
   // CTA's segment list (at most one entry per token) fits
-  if (indexer_group(bt) == 1 && bt->num_q <= IdxDecCfg<HI, DIN, false>::MAXSEG)
-    return fp8 ? launch_indexer_decode<HI, DIN, true>(bt, in, scores, ld, st, pdl)
-               : launch_indexer_decode<HI, DIN, false>(bt, in, scores, ld, st, pdl);
-  if (indexer_group(bt) == 4)
-    return fp8 ? launch_indexer_t<HI, DIN, 4, true>(bt, in, scores, ld, st, pdl)
-               : launch_indexer_t<HI, DIN, 4, false>(bt, in, scores, ld, st, pdl);
-  return fp8 ? launch_indexer_t<HI, DIN, 1, true>(bt, in, scores, ld, st, pdl)
-             : launch_indexer_t<HI, DIN, 1, false>(bt, in, scores, ld, st, pdl);
+  if (indexer_group(bt) == 1 && bt->num_q <= IdxDecCfg<HI, DIN, KF_BF16>::MAXSEG) {
+    if (kf == KF_MX) return launch_indexer_decode<HI, DIN, KF_MX>(bt, in, scores, ld, st, pdl);
+    if (kf == KF_FP8) return launch_indexer_decode<HI, DIN, KF_FP8>(bt, in, scores, ld, st, pdl);
+    return launch_indexer_decode<HI, DIN, KF_BF16>(bt, in, scores, ld, st, pdl);
+  }
+  if (indexer_group(bt) == 4) {
+    if (kf == KF_MX) return launch_indexer_t<HI, DIN, 4, KF_MX>(bt, in, scores, ld, st, pdl);
+    if (kf == KF_FP8) return launch_indexer_t<HI, DIN, 4, KF_FP8>(bt, in, scores, ld, st, pdl);
+    return launch_indexer_t<HI, DIN, 4, KF_BF16>(bt, in, scores, ld, st, pdl);
+  }
+  if (kf == KF_MX) return launch_indexer_t<HI, DIN, 1, KF_MX>(bt, in, scores, ld, st, pdl);
+  if (kf == KF_FP8) return launch_indexer_t<HI, DIN, 1, KF_FP8>(bt, in, scores, ld, st, pdl);
+  return launch_indexer_t<HI, DIN, 1, KF_BF16>(bt, in, scores, ld, st, pdl);
 }
 
 // pdl: launch with programmatic stream serialization, so the prologue may
 // overlap the tail of the previous kernel in the stream (the kernel itself
 // still completes only after that kernel, see its teardown).
-dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_in* in, float* scores, int64_t ld,
-                          cudaStream_t st, bool pdl = false) {
+// Bytes of the widened (bf16) MXFP8 queries in a workspace.
+size_t mx_q_bytes(int T, int h_i, int d_i) { return align256(static_cast<size_t>(T) * h_i * d_i * 2); }
+
+// q_ws: MXFP8 calls only, mx_q_bytes() of 16-byte aligned workspace that
+// receives the widened queries (exact in bf16) before the scoring kernel.
+dsa_status launch_indexer(const dsa_batch* bt, const dsa_indexer_in* in_, float* scores, int64_t ld,
+                          cudaStream_t st, bool pdl = false, void* q_ws = nullptr) {
+  dsa_indexer_in local = *in_;
+  const dsa_indexer_in* in = &local;
+  if (in_->key_dtype == DSA_KEY_MXFP8) {
+    const int64_t n = static_cast<int64_t>(bt->num_q) * in_->n_heads * in_->head_dim;
+    const int64_t blocks64 = (n / 4 + 255) / 256;
+    const int blocks = static_cast<int>(blocks64 < num_sms() * 32 ? blocks64 : num_sms() * 32);
+    mx_dequantize_kernel<<<blocks, 256, 0, st>>>(static_cast<const uint8_t*>(in_->q), in_->q_scale_e8m0, n,
+                                                 static_cast<__nv_bfloat16*>(q_ws));
+    dsa_status s = check_launch("mx_dequantize (queries)");
+    if (s != DSA_OK) return s;
+    local.q = q_ws;
+    pdl = false;  // the scoring kernel reads the queries that kernel writes
+  }
   if (in->n_heads == 64 && in->head_dim == 128) return launch_indexer_g<64, 128>(bt, in, scores, ld, st, pdl);
   if (in->n_heads == 64 && in->head_dim == 32) return launch_indexer_g<64, 32>(bt, in, scores, ld, st, pdl);
   if (in->n_heads == 4 && in->head_dim == 128) return launch_indexer_g<4, 128>(bt, in, scores, ld, st, pdl);
@@ -478,11 +532,11 @@ dsa_status launch_topk(const dsa_batch* bt, const float* scores, int64_t ld, int
   return launch_topk_kernel(topk_kernel<kTopkThreads>, kTopkThreads, cap * 4, p, bt->num_q, st, pdl);
 }
 
-template <int D, int DC>
+template <int D, int DC, bool FP8KV = false>
 dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
                         float* lse, void* ws, size_t ws_bytes, cudaStream_t st, const MlaPlan& pl, bool pdl) {
   using C = MlaCfg<D, DC>;
-  auto kern = sparse_mla_kernel<D, DC>;
+  auto kern = sparse_mla_kernel<D, DC, FP8KV>;
   dsa_status s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   const int T = bt->num_q, H = in->n_heads;
@@ -536,8 +590,7 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  const cudaError_t e =
-      cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(in->kv), qmap, p);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, in->kv, qmap, p);
   if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla launch: %s", cudaGetErrorString(e));
   return check_launch("sparse_mla");
 }
@@ -550,7 +603,7 @@ int pipe_max_clusters(int size, int fallback) {
   if (cache[size] == 0) {
     int n = 0;
     // (no error message is recorded here: a size query may run without a device)
-    if (cudaFuncSetAttribute(sparse_mla_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(sparse_mla_pipe_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              PipeCfg::SMEM_BYTES) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(size, 1, 1);
@@ -563,7 +616,7 @@ int pipe_max_clusters(int size, int fallback) {
       attr.val.clusterDim.z = 1;
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
-      if (cudaOccupancyMaxActiveClusters(&n, sparse_mla_pipe_kernel, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, sparse_mla_pipe_kernel<false>, &cfg) != cudaSuccess) n = 0;
     }
     cudaGetLastError();  // clear a failed query's error state
     cache[size] = n > 0 ? n : -1;
@@ -574,7 +627,8 @@ int pipe_max_clusters(int size, int fallback) {
 dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
                            float* lse, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl) {
   using C = PipeCfg;
-  dsa_status s = set_smem(sparse_mla_pipe_kernel, C::SMEM_BYTES);
+  auto kern = bt->block_table ? sparse_mla_pipe_kernel<true> : sparse_mla_pipe_kernel<false>;
+  dsa_status s = set_smem(kern, C::SMEM_BYTES);
   if (s != DSA_OK) return s;
   const int T = bt->num_q;
   const MlaPlan pl = pipe_plan(T, k, num_sms());
@@ -649,7 +703,7 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
   cfg.attrs = attr;
   cfg.numAttrs = na;
   const cudaError_t e =
-      cudaLaunchKernelEx(&cfg, sparse_mla_pipe_kernel, kvmap, qmap, pmap, p);
+      cudaLaunchKernelEx(&cfg, kern, kvmap, qmap, pmap, p);
   if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "sparse_mla_pipe launch: %s", cudaGetErrorString(e));
   return check_launch("sparse_mla_pipe");
 }
@@ -657,6 +711,15 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
 dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out, float* lse,
                       void* ws, size_t ws_bytes, cudaStream_t st, bool pdl = false) {
   const int hb = (in->n_heads + 63) / 64;
+  if (in->kv_dtype == DSA_KV_FP8_E4M3) {
+    // FP8 rows: the one-CTA-per-head-block kernel widens them on chip
+    if (in->d_latent == 512) {
+      const MlaPlan pl = mla_plan(bt->num_q, hb, k, num_sms(), MlaCfg<576, 512>::TK);
+      return launch_mla_t<576, 512, true>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
+    }
+    const MlaPlan pl = mla_plan(bt->num_q, hb, k, num_sms(), MlaCfg<80, 64>::TK);
+    return launch_mla_t<80, 64, true>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
+  }
   if (in->d_latent == 512 && in->n_heads == PipeCfg::M && bt->num_q <= 65535)  // queries on grid y
     return launch_mla_pipe(bt, in, idx, k, out, lse, ws, ws_bytes, st, pdl);
   if (in->d_latent == 512) {
@@ -693,20 +756,19 @@ const char* dsa_status_string(dsa_status s) {
 const char* dsa_last_error(void) { return g_last_error; }
 
 size_t dsa_workspace_size(int op, const dsa_batch* batch, int32_t k, int32_t h_i, int32_t d_i) {
-  (void)h_i;
-  (void)d_i;
-  if (!batch || batch->num_q <= 0 || k <= 0) return 0;
+  if (!batch || batch->num_q <= 0) return 0;
   const int T = batch->num_q;
-  const int sms = num_sms();
+  const size_t qb = (h_i > 0 && d_i > 0) ? mx_q_bytes(T, h_i, d_i) : 0;
+  if (op == DSA_OP_INDEXER_SCORES) return qb;
+  if (k <= 0) return 0;
   switch (op) {
-    case DSA_OP_INDEXER_SCORES:
     case DSA_OP_TOPK:
       return 0;
     case DSA_OP_SPARSE_MLA:
       return mla_ws_bytes(batch, k);
     case DSA_OP_FUSED_DECODE:
       return align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float)) +
-             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes(batch, k);
+             align256(static_cast<size_t>(T) * k * sizeof(int32_t)) + mla_ws_bytes(batch, k) + qb;
     default:
       return 0;
   }
@@ -714,15 +776,18 @@ size_t dsa_workspace_size(int op, const dsa_batch* batch, int32_t k, int32_t h_i
 
 dsa_status dsa_indexer_scores(const dsa_batch* batch, const dsa_indexer_in* in, float* scores, int64_t score_ld,
                               void* ws, size_t ws_bytes, dsa_stream_t stream) {
-  (void)ws;
-  (void)ws_bytes;
   dsa_status s = check_batch(batch);
   if (s != DSA_OK) return s;
   if ((s = check_indexer(batch, in)) != DSA_OK) return s;
   if (!scores) return fail(DSA_ERR_INVALID_ARGUMENT, "scores is NULL");
   if (score_ld < batch->max_seq_len) return fail(DSA_ERR_INVALID_ARGUMENT, "score_ld < max_seq_len");
   if (batch->num_q == 0) return DSA_OK;
-  return launch_indexer(batch, in, scores, score_ld, reinterpret_cast<cudaStream_t>(stream));
+  if (in->key_dtype == DSA_KEY_MXFP8) {
+    const size_t need = mx_q_bytes(batch->num_q, in->n_heads, in->head_dim);
+    if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
+    if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+  }
+  return launch_indexer(batch, in, scores, score_ld, reinterpret_cast<cudaStream_t>(stream), false, ws);
 }
 
 dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t score_ld, int32_t k, int32_t* idx,
@@ -766,7 +831,8 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
   const size_t sc_bytes = align256(static_cast<size_t>(T) * batch->max_seq_len * sizeof(float));
   const size_t id_bytes = align256(static_cast<size_t>(T) * k * sizeof(int32_t));
   const size_t mla_bytes = mla_ws_bytes(batch, k);
-  const size_t need = sc_bytes + id_bytes + mla_bytes;
+  const size_t q_bytes = idx_in->key_dtype == DSA_KEY_MXFP8 ? mx_q_bytes(T, idx_in->n_heads, idx_in->head_dim) : 0;
+  const size_t need = sc_bytes + id_bytes + mla_bytes + q_bytes;
   if (!ws || ws_bytes < need) return fail(DSA_ERR_WORKSPACE_TOO_SMALL, "workspace %zu < %zu bytes", ws_bytes, need);
   if (!aligned16(ws)) return fail(DSA_ERR_MISALIGNED, "workspace must be 16-byte aligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -783,7 +849,9 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
   // when stage events sit between the kernels.
   const bool pdl = stage_events == nullptr;
   if ((s = rec(0)) != DSA_OK) return s;
-  if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st, pdl)) != DSA_OK) return s;
+  if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st, pdl,
+                          static_cast<uint8_t*>(ws) + sc_bytes + id_bytes + mla_bytes)) != DSA_OK)
+    return s;
   if ((s = rec(1)) != DSA_OK) return s;
   if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st, pdl)) != DSA_OK) return s;
   if ((s = rec(2)) != DSA_OK) return s;
@@ -815,6 +883,49 @@ dsa_status dsa_quantize_index_keys(const void* k_bf16, int64_t n_keys, int32_t d
   else
     quantize_keys_kernel<128><<<blocks, 256, 0, st>>>(k, n_keys, dim, k8, scale);
   return check_launch("quantize_index_keys");
+}
+
+dsa_status dsa_quantize_mxfp8(const void* x_bf16, int64_t n_rows, int32_t dim, uint8_t* codes, uint8_t* scales,
+                              dsa_stream_t stream) {
+  if (!x_bf16 || !codes || !scales) return fail(DSA_ERR_INVALID_ARGUMENT, "x_bf16, codes, scales must be non-NULL");
+  if (n_rows < 0) return fail(DSA_ERR_INVALID_ARGUMENT, "n_rows < 0");
+  if (dim <= 0 || dim > 1024 || dim % 32 != 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "dim %d must be a multiple of 32 and <= 1024", dim);
+  if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales))
+    return fail(DSA_ERR_MISALIGNED, "x_bf16, codes, scales must be 16-byte aligned");
+  if (n_rows == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+  const int64_t blocks64 = (n_rows + 7) / 8;
+  const int blocks = static_cast<int>(blocks64 < sms * 16 ? blocks64 : sms * 16);
+  mx_quantize_kernel<<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x_bf16), n_rows, dim, codes, scales);
+  return check_launch("quantize_mxfp8");
+}
+
+size_t dsa_kv_fp8_row_bytes(int32_t d_latent, int32_t d_rope) {
+  if (d_latent == 512 && d_rope == 64) return KvFp8Row<512, 64>::ROW_BYTES;
+  if (d_latent == 64 && d_rope == 16) return KvFp8Row<64, 16>::ROW_BYTES;
+  return 0;
+}
+
+dsa_status dsa_quantize_kv(const void* kv_bf16, int64_t n_rows, int32_t d_latent, int32_t d_rope, uint8_t* kv_fp8,
+                           dsa_stream_t stream) {
+  if (!kv_bf16 || !kv_fp8) return fail(DSA_ERR_INVALID_ARGUMENT, "kv_bf16 and kv_fp8 must be non-NULL");
+  if (n_rows < 0) return fail(DSA_ERR_INVALID_ARGUMENT, "n_rows < 0");
+  if (dsa_kv_fp8_row_bytes(d_latent, d_rope) == 0)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "KV dims (%d,%d) not in {(512,64),(64,16)}", d_latent, d_rope);
+  if (!aligned16(kv_bf16) || !aligned16(kv_fp8)) return fail(DSA_ERR_MISALIGNED, "kv_bf16 and kv_fp8 must be 16-byte aligned");
+  if (n_rows == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+  const int64_t blocks64 = (n_rows + 7) / 8;
+  const int blocks = static_cast<int>(blocks64 < sms * 16 ? blocks64 : sms * 16);
+  const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(kv_bf16);
+  if (d_latent == 512)
+    quantize_kv_kernel<512, 64><<<blocks, 256, 0, st>>>(kv, n_rows, kv_fp8);
+  else
+    quantize_kv_kernel<64, 16><<<blocks, 256, 0, st>>>(kv, n_rows, kv_fp8);
+  return check_launch("quantize_kv");
 }
 
 dsa_status dsa_dequantize_index_keys(const uint8_t* k8, const float* scale, int64_t n_keys, int32_t dim,
@@ -953,8 +1064,12 @@ dsa_status noalloc_scratch(void** out) {
 dsa_status launch_mla_unsplit(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* idx, int k, void* out,
                               float* lse, cudaStream_t st) {
   const MlaPlan pl{1, ((k + 63) / 64) * 64};
-  if (in->d_latent == 512) return launch_mla_t<576, 512>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false);
-  return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false);
+  const bool f8 = in->kv_dtype == DSA_KV_FP8_E4M3;
+  if (in->d_latent == 512)
+    return f8 ? launch_mla_t<576, 512, true>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false)
+              : launch_mla_t<576, 512>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false);
+  return f8 ? launch_mla_t<80, 64, true>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false)
+            : launch_mla_t<80, 64>(bt, in, idx, k, out, lse, nullptr, 0, st, pl, false);
 }
 
 }  // namespace
@@ -966,6 +1081,8 @@ extern "C" dsa_status dsa_fused_decode_noalloc(const dsa_batch* batch, const dsa
   if (s != DSA_OK) return s;
   if ((s = check_indexer(batch, idx_in)) != DSA_OK) return s;
   if ((s = check_mla(mla_in)) != DSA_OK) return s;
+  if (idx_in->key_dtype == DSA_KEY_MXFP8)
+    return fail(DSA_ERR_UNSUPPORTED_SHAPE, "dsa_fused_decode_noalloc does not take MXFP8 index inputs");
   if (!out) return fail(DSA_ERR_INVALID_ARGUMENT, "out is NULL");
   if (!aligned16(out) || (idx_out && !aligned16(idx_out)))
     return fail(DSA_ERR_MISALIGNED, "out and idx_out must be 16-byte aligned");

@@ -17,12 +17,19 @@
 // head weights, the FP8 scale and the causal / length mask, and store the
 // scores coalesced. FP8 keys are TMA-loaded as bytes and widened to bf16 in
 // shared memory by four converter warps (exact: every E4M3 value is a bf16).
+// Key formats (KF): 0 BF16; 1 FP8 with one fp32 scale per key (sigma_s
+// above); 2 MXFP8, one power-of-two (E8M0) scale per 32 elements (Index Q/K
+// Uses MXFP8, section 4.2 of "Inference Adaptation and Performance
+// Optimization for New Large Language Model Architectures"), applied by the
+// converters while widening (exact in bf16; sigma_s = 1), its scale bytes
+// copied into the stage with the codes when their rows are 16-byte aligned.
 //
 // Roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner), then the
 // epilogue warps (four; eight for multi-token groups, two per TMEM
 // sub-partition splitting the tokens), then four FP8 converters (FP8 only).
 #pragma once
 #include "dsa_common.cuh"
+#include "quant.cuh"
 
 namespace dsa {
 
@@ -35,14 +42,19 @@ struct IndexerParams {
   const __nv_bfloat16* q;   // [T, HI, DIN]
   const float* w;           // [T, HI]
   const float* k_scale;     // one scale per cache row (FP8) or null
+  const uint8_t* k_mx;      // MXFP8: E8M0 bytes [cache rows, DIN / 32] or null
+  int32_t scale_bulk;       // MXFP8: scale bytes are copied into the stage (16-byte aligned rows)
+  int64_t rows;             // cache rows (contiguous B * L_max, or the page pool)
   float* scores;            // [T, ld]
   int64_t ld;
   int32_t tiles_per_cta;
   CacheMap cm;              // cache rows (contiguous or paged)
 };
 
-template <int HI, int DIN, int G, bool FP8>
+template <int HI, int DIN, int G, int KF>
 struct IndexerCfg {
+  static constexpr bool FP8 = KF != 0;                     // 8-bit codes (FP8 or MXFP8), widened on chip
+  static constexpr int SROW = KF == 2 ? DIN / 32 : 0;      // MXFP8 scale bytes per key row (staged)
   static constexpr int DK = DIN < 64 ? 64 : DIN;           // K padded to whole 128-byte atoms
   static constexpr int AK = DK / 64;                       // atom columns along K
   static constexpr int N = ((G * HI + 15) / 16) * 16;      // MMA N
@@ -64,7 +76,7 @@ struct IndexerCfg {
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_STAGE = OFF_Q + ((Q_BYTES + 1023) / 1024) * 1024;
-  static constexpr int STAGE_BYTES = FP8 ? U8_TILE : TILE_BYTES;
+  static constexpr int STAGE_BYTES = FP8 ? U8_TILE + 128 * SROW : TILE_BYTES;
   static constexpr int OFF_CONV = OFF_STAGE + ((ST * STAGE_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_BAR = OFF_CONV + (FP8 ? CS * TILE_BYTES : 0);
   static constexpr int NUM_BARS = 2 * ST + 2 * NACC + 2 * CS + 1;
@@ -79,10 +91,11 @@ struct IndexerCfg {
   static_assert(ST >= 2, "need at least two stages");
 };
 
-template <int HI, int DIN, int G, bool FP8>
-__global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerCfg<HI, DIN, G, FP8>::MIN_CTAS)
+template <int HI, int DIN, int G, int KF>
+__global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCfg<HI, DIN, G, KF>::MIN_CTAS)
     indexer_scores_kernel(const __grid_constant__ CUtensorMap kmap, const IndexerParams p) {
-  using C = IndexerCfg<HI, DIN, G, FP8>;
+  using C = IndexerCfg<HI, DIN, G, KF>;
+  constexpr bool FP8 = C::FP8;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-byte alignment
@@ -217,23 +230,32 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
     const int st = it % C::ST;
     const int s0 = (tile_begin + it) * 128;  // first key position of the tile
     const uint32_t dst = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES);
-    mbar_arrive_expect_tx(&full[st], FP8 ? C::U8_TILE : C::TILE_BYTES);
     if (!p.cm.paged()) {
       const int32_t y = static_cast<int32_t>(row0 + s0);
       if constexpr (FP8) {
+        // MXFP8: scale rows y .. y + 127, clipped at the end of the cache
+        const int64_t left = p.rows - y;
+        const uint32_t sbytes = (C::SROW && p.scale_bulk) ? C::SROW * static_cast<uint32_t>(left < 128 ? left : 128) : 0u;
+        mbar_arrive_expect_tx(&full[st], C::U8_TILE + sbytes);
         tma_load_2d(dst, &kmap, 0, y, &full[st]);
+        if (sbytes) bulk_load(dst + C::U8_TILE, p.k_mx + static_cast<int64_t>(y) * C::SROW, sbytes, &full[st]);
       } else {
+        mbar_arrive_expect_tx(&full[st], C::TILE_BYTES);
 #pragma unroll
         for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384, &kmap, a * 64, y, &full[st]);
       }
     } else {
       // paged: two 64-row boxes (a page holds a whole number of them); a half
       // past the last candidate reloads the first half (its rows are masked)
+      mbar_arrive_expect_tx(&full[st], FP8 ? C::U8_TILE + (p.scale_bulk ? 128 * C::SROW : 0) : C::TILE_BYTES);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int32_t y = p.cm.row_checked(b, (s0 + 64 * h < nk) ? s0 + 64 * h : s0);
         if constexpr (FP8) {
           tma_load_2d(dst + h * 64 * DIN, &kmap, 0, y, &full[st]);
+          if (C::SROW && p.scale_bulk)
+            bulk_load(dst + C::U8_TILE + 64 * C::SROW * h, p.k_mx + static_cast<int64_t>(y) * C::SROW, 64 * C::SROW,
+                      &full[st]);
         } else {
 #pragma unroll
           for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384 + h * 8192, &kmap, a * 64, y, &full[st]);
@@ -418,7 +440,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       const int64_t s = static_cast<int64_t>(tile_begin + it) * 128 + r;
       float sigma = 1.0f;
-      if constexpr (FP8) {
+      if constexpr (KF == 1) {
         if (s < nk) {
           bool ok;
           const int32_t kr = p.cm.row(b, static_cast<int>(s), ok);
@@ -445,20 +467,52 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, FP8>::THREADS, IndexerC
       const int cs = it % C::CS;
       if (!mbar_wait(&full[st], (it / C::ST) & 1, abort_flag)) break;
       if (!mbar_wait(&conv_empty[cs], ((it / C::CS) & 1) ^ 1, abort_flag)) break;
-      const uint8_t* src = smem + C::OFF_STAGE + st * C::U8_TILE;
+      const uint8_t* src = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
       uint8_t* dst = smem + C::OFF_CONV + cs * C::TILE_BYTES;
-      for (int i = ct; i < 128 * CPR; i += 128) {
+      const int s0 = (tile_begin + it) * 128;  // first key position of the tile
+      // all of the thread's chunks (and MXFP8 scale bytes) are loaded first
+      constexpr int PER = (128 * CPR + 127) / 128;
+      uint4 raws[PER];
+      int bytes[PER];
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int i = ct + u * 128;
         const int row = i / CPR;
         const int c = i % CPR;
-        const uint4 raw = *reinterpret_cast<const uint4*>(src + row * DIN + c * 16);
-        const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+        raws[u] = *reinterpret_cast<const uint4*>(src + row * DIN + c * 16);
+        bytes[u] = 127;
+        if constexpr (KF == 2) {
+          if (p.scale_bulk) {
+            bytes[u] = src[C::U8_TILE + row * (DIN / 32) + c / 2];
+          } else {
+            // rows past the last candidate are masked; read a row that exists
+            bool rok;
+            const int sr = s0 + row < nk ? s0 + row : s0;
+            bytes[u] = __ldg(p.k_mx + static_cast<int64_t>(p.cm.row(b, sr, rok)) * (DIN / 32) + c / 2);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < PER; ++u) {
+        const int i = ct + u * 128;
+        const int row = i / CPR;
+        const int c = i % CPR;
+        const uint32_t words[4] = {raws[u].x, raws[u].y, raws[u].z, raws[u].w};
+        // MXFP8: 2^e of the chunk's 32-element group (exact scaling)
+        const float m = KF == 2 ? exp2_int(bytes[u] - 127) : 1.0f;
         uint32_t outw[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const __half2_raw h01 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(words[q] & 0xFFFF), __NV_E4M3);
           const __half2_raw h23 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(words[q] >> 16), __NV_E4M3);
-          const float2 f01 = __half22float2(__half2(h01));
-          const float2 f23 = __half22float2(__half2(h23));
+          float2 f01 = __half22float2(__half2(h01));
+          float2 f23 = __half22float2(__half2(h23));
+          if constexpr (KF == 2) {
+            f01.x *= m;
+            f01.y *= m;
+            f23.x *= m;
+            f23.y *= m;
+          }
           const __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
           const __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
           outw[2 * q] = *reinterpret_cast<const uint32_t*>(&b01);

@@ -19,13 +19,19 @@
 // buffers, and per key tile a TMA load into one of ST stages. Warp 1 issues
 // tcgen05.mma with M = 128 keys, N = heads, K = d_I into two TMEM
 // accumulators. Four epilogue warps read one key row per thread, apply ReLU,
-// the weights, the key's scale (FP8; read from global memory by the thread
-// that owns the row) and the causal / length mask and store the scores. FP8
-// codes are widened to bf16 by four converter warps (exact: every E4M3 value
-// is a bf16), which free the stage once its codes are converted. Every wait
-// is bounded.
+// the weights, the key's scale (FP8) and the causal / length mask and store
+// the scores. FP8 codes are widened to bf16 by four converter warps (exact:
+// every E4M3 value is a bf16). Key formats (KF): BF16; FP8 with one fp32 scale
+// per key, applied after the head sum; MXFP8 with one power-of-two (E8M0)
+// scale per 32 elements, applied by the converters while widening (still
+// exact in bf16), with queries given in bf16 (the host widens MXFP8 queries
+// first). A tile's scales ride in its stage (one bulk copy per 64 or 128
+// rows) when the scale rows are 16-byte aligned; otherwise each reader loads
+// them from global memory. FP8 / MXFP8 stages are freed by the epilogue,
+// after every reader of the stage is done. Every wait is bounded.
 #pragma once
 #include "dsa_common.cuh"
+#include "quant.cuh"
 
 namespace dsa {
 
@@ -33,7 +39,10 @@ struct IdxDecParams {
   const int32_t* cu_q;
   const int32_t* q_pos;
   const int32_t* seq_lens;
-  const float* k_scale;  // FP8 keys: one scale per cache row
+  const float* k_scale;     // FP8 keys: one fp32 scale per cache row
+  const uint8_t* k_mx;      // MXFP8 keys: E8M0 bytes [cache rows, d_I / 32]
+  int32_t scale_bulk;       // scales are copied into the stage (16-byte aligned rows)
+  int64_t rows;          // cache rows (contiguous B * L_max, or the page pool)
   int32_t B;
   int32_t T;
   int32_t L_max;
@@ -42,14 +51,19 @@ struct IdxDecParams {
   CacheMap cm;    // cache rows (contiguous or paged)
 };
 
-template <int HI, int DIN, bool FP8>
+// Key formats of the indexer kernels.
+constexpr int KF_BF16 = 0, KF_FP8 = 1, KF_MX = 2;
+
+template <int HI, int DIN, int KF>
 struct IdxDecCfg {
+  static constexpr bool FP8 = KF != KF_BF16;             // 8-bit codes, widened by converter warps
+  static constexpr int SROW = KF == KF_FP8 ? 4 : KF == KF_MX ? DIN / 32 : 0;  // scale bytes per key row
   static constexpr int DK = DIN < 64 ? 64 : DIN;         // K padded to whole 128-byte atoms
   static constexpr int AK = DK / 64;                     // atom columns along K
   static constexpr int N = ((HI + 15) / 16) * 16;        // MMA N (zero rows beyond HI)
   static constexpr int TILE_BYTES = 128 * DK * 2;        // bf16 key tile (A operand)
   static constexpr int U8_TILE = 128 * DIN;              // FP8 codes of a tile
-  static constexpr int STAGE_BYTES = FP8 ? U8_TILE : TILE_BYTES;
+  static constexpr int STAGE_BYTES = FP8 ? U8_TILE + 128 * SROW : TILE_BYTES;  // codes + the tile's scales
   static constexpr int ST = FP8 ? 6 : 5;                 // key stages
   static constexpr int CS = 2;                           // converted bf16 tiles (FP8)
   static constexpr int NACC = 2;                         // TMEM accumulators
@@ -59,7 +73,8 @@ struct IdxDecCfg {
   static constexpr int W_BYTES = ((HI * 4 + 15) / 16) * 16;
   static constexpr int MAXSEG = 256;                     // segments a CTA can hold (tokens <= MAXSEG)
   static constexpr int EPI_WARPS = 4;
-  static constexpr int NUM_WARPS = 2 + EPI_WARPS + (FP8 ? 4 : 0);
+  static constexpr int CONV_WARPS = FP8 ? 8 : 0;         // FP8 -> bf16 converters (two per SM sub-partition)
+  static constexpr int NUM_WARPS = 2 + EPI_WARPS + CONV_WARPS;
   static constexpr int THREADS = NUM_WARPS * 32;
   // shared memory (offsets from the 1024-byte-aligned window)
   static constexpr int OFF_Q = 0;
@@ -78,19 +93,20 @@ struct IdxDecCfg {
   static_assert(N <= 256, "MMA N");
 };
 
-template <int HI, int DIN, bool FP8>
-__global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
+template <int HI, int DIN, int KF>
+__global__ void __launch_bounds__(IdxDecCfg<HI, DIN, KF>::THREADS, 1)
     indexer_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                           const float* __restrict__ w, const IdxDecParams p) {
-  using C = IdxDecCfg<HI, DIN, FP8>;
+  using C = IdxDecCfg<HI, DIN, KF>;
+  constexpr bool FP8 = C::FP8;
   extern __shared__ __align__(1024) uint8_t smem[];
   if (smem_u32(smem) & 1023u) {  // swizzled tiles need 1024-byte alignment (same in every CTA)
     if (threadIdx.x == 0) set_device_status(DSA_ERR_DEVICE_LAYOUT);
     return;
   }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* full = bars;                       // [ST]   producer -> MMA (BF16) or converters (FP8)
-  uint64_t* empty = full + C::ST;              // [ST]   MMA (BF16) or converters (FP8) -> producer
+  uint64_t* full = bars;                       // [ST]   producer -> MMA (BF16) or converters + epilogue (FP8)
+  uint64_t* empty = full + C::ST;              // [ST]   MMA (BF16) or epilogue (FP8) -> producer
   uint64_t* acc_full = empty + C::ST;          // [NACC] MMA -> epilogue
   uint64_t* acc_empty = acc_full + C::NACC;    // [NACC] epilogue -> MMA
   uint64_t* conv_full = acc_empty + C::NACC;   // [CS]   converters -> MMA
@@ -186,14 +202,14 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
       misc[3] = static_cast<int>(hi - lo);
       for (int i = 0; i < C::ST; ++i) {
         mbar_init(&full[i], 1);
-        mbar_init(&empty[i], FP8 ? 4 : 1);
+        mbar_init(&empty[i], FP8 ? C::EPI_WARPS : 1);
       }
       for (int i = 0; i < C::NACC; ++i) {
         mbar_init(&acc_full[i], 1);
         mbar_init(&acc_empty[i], C::EPI_WARPS);
       }
       for (int i = 0; i < C::CS; ++i) {
-        mbar_init(&conv_full[i], 4);
+        mbar_init(&conv_full[i], C::CONV_WARPS);
         mbar_init(&conv_empty[i], 1);
       }
       for (int i = 0; i < 2; ++i) {
@@ -230,6 +246,7 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
     if (warp == 0) {
       // ---------------------------------------------------------- producer
       if (lane == 0) {
+        const uint8_t* scale_src = KF == KF_MX ? p.k_mx : reinterpret_cast<const uint8_t*>(p.k_scale);
         int it = 0, kq = 0;
         bool ok = true;
         for (int k = 0; k < nseg && ok; ++k) {
@@ -253,23 +270,33 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
             }
             const int s0 = (seg_t0[k] + i) * 128;  // first key position of the tile
             const uint32_t dst = smem_u32(smem + C::OFF_STAGE + st * C::STAGE_BYTES);
-            mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
             if (!p.cm.paged()) {
               const int32_t y = bb * p.L_max + s0;
               if constexpr (FP8) {
+                // scale rows y .. y + 127, clipped at the end of the cache
+                const int64_t left = p.rows - y;
+                const uint32_t sbytes =
+                    p.scale_bulk ? C::SROW * static_cast<uint32_t>(left < 128 ? left : 128) : 0u;
+                mbar_arrive_expect_tx(&full[st], C::U8_TILE + sbytes);
                 tma_load_2d(dst, &kmap, 0, y, &full[st]);
+                if (sbytes) bulk_load(dst + C::U8_TILE, scale_src + static_cast<int64_t>(y) * C::SROW, sbytes, &full[st]);
               } else {
+                mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
 #pragma unroll
                 for (int a = 0; a < C::AK; ++a) tma_load_2d(dst + a * 16384, &kmap, a * 64, y, &full[st]);
               }
             } else {
               // paged: two 64-row boxes; a half past the last candidate
               // reloads the first half (its rows are masked)
+              mbar_arrive_expect_tx(&full[st], FP8 ? C::U8_TILE + (p.scale_bulk ? 128 * C::SROW : 0) : C::STAGE_BYTES);
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
                 const int32_t y = p.cm.row_checked(bb, (s0 + 64 * h < nv) ? s0 + 64 * h : s0);
                 if constexpr (FP8) {
                   tma_load_2d(dst + h * 64 * DIN, &kmap, 0, y, &full[st]);
+                  if (p.scale_bulk)
+                    bulk_load(dst + C::U8_TILE + 64 * C::SROW * h, scale_src + static_cast<int64_t>(y) * C::SROW,
+                              64 * C::SROW, &full[st]);
                 } else {
 #pragma unroll
                   for (int a = 0; a < C::AK; ++a)
@@ -352,14 +379,21 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
           const int64_t s = static_cast<int64_t>(seg_t0[k] + i) * 128 + r;  // key position of this row
           float sigma = 1.0f;
           if constexpr (FP8) {
-            // the key's scale, loaded while the MMA runs (only rows that
-            // are causal candidates, so only inside the sequence's rows)
-            if (s < nv) {
+            // the stage (codes + scales) stays ours until this warp frees it
+            const int st = it % C::ST;
+            ok = mbar_wait_warp(&full[st], (it / C::ST) & 1, abort_flag);
+            if constexpr (KF != KF_FP8) {
+              // MXFP8: the scales were applied while widening
+            } else if (p.scale_bulk) {
+              if (ok) sigma = reinterpret_cast<const float*>(smem + C::OFF_STAGE + st * C::STAGE_BYTES + C::U8_TILE)[r];
+            } else if (s < nv) {
+              // the key's scale from global memory (only causal candidates,
+              // so only rows inside the sequence)
               bool rok;
               sigma = __ldg(p.k_scale + p.cm.row(bb, static_cast<int>(s), rok));
             }
           }
-          ok = mbar_wait_warp(&acc_full[acc], (it / C::NACC) & 1, abort_flag);
+          if (ok) ok = mbar_wait_warp(&acc_full[acc], (it / C::NACC) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           float score;
@@ -392,7 +426,10 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[acc]);
+          if (lane == 0) {
+            mbar_arrive(&acc_empty[acc]);
+            if constexpr (FP8) mbar_arrive(&empty[it % C::ST]);  // codes converted, scales read
+          }
           if (s < p.ld) p.scores[static_cast<int64_t>(t) * p.ld + s] = (s < nv) ? score * sigma : -INFINITY;
         }
         __syncwarp();
@@ -400,11 +437,16 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
       }
     } else if constexpr (FP8) {
       // ---------------------------------------------------------- FP8 -> bf16 converters
-      const int ct = threadIdx.x - (2 + C::EPI_WARPS) * 32;  // 0..127
+      // Each thread loads all its 16-byte code chunks of the tile first (and,
+      // for MXFP8, their scale bytes), then widens and stores them.
+      constexpr int CT = C::CONV_WARPS * 32;
+      const int ct = threadIdx.x - (2 + C::EPI_WARPS) * 32;  // 0 .. CT - 1
       constexpr int CPR = DIN / 16;                            // 16-byte code chunks per key row
+      constexpr int PER = (128 * CPR + CT - 1) / CT;           // chunks per thread
       int it = 0;
       bool ok = true;
       for (int k = 0; k < nseg && ok; ++k) {
+        const int bb = seg_b[k];
         for (int i = 0; i < seg_nt[k]; ++i, ++it) {
           const int st = it % C::ST;
           const int cs = it % C::CS;
@@ -413,11 +455,39 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
           if (!ok) break;
           const uint8_t* src = smem + C::OFF_STAGE + st * C::STAGE_BYTES;
           uint8_t* dst = smem + C::OFF_CONV + cs * C::TILE_BYTES;
-          for (int e = ct; e < 128 * CPR; e += 128) {
+          const int s0 = (seg_t0[k] + i) * 128;  // first key position of the tile
+          uint4 raws[PER];
+          int bytes[PER];
+#pragma unroll
+          for (int u = 0; u < PER; ++u) {
+            const int e = ct + u * CT;
             const int row = e / CPR;
             const int c = e % CPR;
-            const uint4 raw = *reinterpret_cast<const uint4*>(src + row * DIN + c * 16);
-            const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+            raws[u] = make_uint4(0u, 0u, 0u, 0u);
+            bytes[u] = 127;
+            if (e < 128 * CPR) {
+              raws[u] = *reinterpret_cast<const uint4*>(src + row * DIN + c * 16);
+              if constexpr (KF == KF_MX) {
+                if (p.scale_bulk) {
+                  bytes[u] = src[C::U8_TILE + row * (DIN / 32) + c / 2];
+                } else {
+                  // rows past the sequence are masked; read a row that exists
+                  bool rok;
+                  const int sr = s0 + row < seg_nv[k] ? s0 + row : s0;
+                  bytes[u] = __ldg(p.k_mx + static_cast<int64_t>(p.cm.row(bb, sr, rok)) * (DIN / 32) + c / 2);
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < PER; ++u) {
+            const int e = ct + u * CT;
+            if (e >= 128 * CPR) break;
+            const int row = e / CPR;
+            const int c = e % CPR;
+            const uint32_t words[4] = {raws[u].x, raws[u].y, raws[u].z, raws[u].w};
+            // MXFP8: 2^e of the chunk's 32-element group (exact scaling)
+            const float m = KF == KF_MX ? exp2_int(bytes[u] - 127) : 1.0f;
             uint32_t outw[8];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -425,8 +495,15 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
                   __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(words[q] & 0xFFFF), __NV_E4M3);
               const __half2_raw h23 =
                   __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(words[q] >> 16), __NV_E4M3);
-              const __nv_bfloat162 b01 = __float22bfloat162_rn(__half22float2(__half2(h01)));
-              const __nv_bfloat162 b23 = __float22bfloat162_rn(__half22float2(__half2(h23)));
+              float2 f01 = __half22float2(__half2(h01)), f23 = __half22float2(__half2(h23));
+              if constexpr (KF == KF_MX) {
+                f01.x *= m;
+                f01.y *= m;
+                f23.x *= m;
+                f23.y *= m;
+              }
+              const __nv_bfloat162 b01 = __float22bfloat162_rn(f01);
+              const __nv_bfloat162 b23 = __float22bfloat162_rn(f23);
               outw[2 * q] = *reinterpret_cast<const uint32_t*>(&b01);
               outw[2 * q + 1] = *reinterpret_cast<const uint32_t*>(&b23);
             }
@@ -439,10 +516,7 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, FP8>::THREADS, 1)
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&conv_full[cs]);
-            mbar_arrive(&empty[st]);  // the codes are converted: the stage may be refilled
-          }
+          if (lane == 0) mbar_arrive(&conv_full[cs]);
         }
       }
     }

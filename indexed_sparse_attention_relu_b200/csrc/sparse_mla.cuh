@@ -40,6 +40,7 @@
 // Every wait is bounded.
 #pragma once
 #include "dsa_common.cuh"
+#include "quant.cuh"
 
 namespace dsa {
 
@@ -165,11 +166,35 @@ __device__ __forceinline__ void q_pair(uint32_t q_stage, int ha, int hbr, int co
   xb1 = y.y;
 }
 
-template <int D, int DC>
+// FP8 latent rows: widen 16 E4M3 codes (one 16-byte chunk) times their tile
+// scale to 16 bf16 values (two 16-byte chunks), rounding fl32(code * s) to
+// nearest bf16; the tensor cores then see bf16 as for bf16 caches.
+__device__ __forceinline__ void fp8x16_to_bf16x16(const uint4& raw, float s, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const __half2_raw hr =
+          __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>((w[q] >> (16 * h)) & 0xFFFFu), __NV_E4M3);
+      float2 f = __half22float2(__half2(hr));
+      f.x *= s;
+      f.y *= s;
+      const __nv_bfloat162 b = __float22bfloat162_rn(f);
+      o[2 * q + h] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <int D, int DC, bool FP8KV = false>
 __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
-    sparse_mla_kernel(const __nv_bfloat16* __restrict__ kv, const __grid_constant__ CUtensorMap qmap,
+    sparse_mla_kernel(const void* __restrict__ kv_ptr, const __grid_constant__ CUtensorMap qmap,
                       const MlaParams p) {
   using C = MlaCfg<D, DC>;
+  const __nv_bfloat16* kv = static_cast<const __nv_bfloat16*>(kv_ptr);
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled tiles need 1024-byte alignment; the dynamic window starts at
   // the same offset in every CTA, so either all CTAs leave here or none.
@@ -253,6 +278,73 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     };
     int nxt = row_index(0);
     bool ok = true;
+    if constexpr (FP8KV) {
+      // FP8 rows (KvFp8Row layout): every lane loads its 16-byte chunks of
+      // the tile (codes with their tile scale, rope chunks) before waiting
+      // for the stage, then widens them into the swizzled bf16 stage and
+      // arrives once the stores are visible to the tensor cores.
+      using R = KvFp8Row<DC, D - DC>;
+      constexpr int CC = DC / 16;               // code chunks per row (16 codes each)
+      constexpr int RC = (D - DC) / 8;          // rope chunks per row (8 bf16 each)
+      constexpr int ZC = (C::DP - D) / 8;       // stored chunks past D (zero)
+      constexpr int IPR = CC + RC + ZC;         // work items per row
+      constexpr int RND = (C::RPW * IPR + 31) / 32;
+      const uint8_t* kv8 = static_cast<const uint8_t*>(kv_ptr);
+      for (int it = 0; it < n_tiles && ok; ++it) {
+        const int sl = it % C::NST;
+        const uint32_t use = static_cast<uint32_t>(it / C::NST);
+        const int cur = nxt;
+        const bool okr = cur >= 0 && cur < len;
+        if (lane < C::RPW && cur != -1 && !okr) set_device_status(DSA_ERR_DEVICE_INDEX);
+        const int mine = okr ? p.cm.row_checked(b, cur) : -1;  // cache row of this lane's key
+        uint4 raw[RND];
+        float sc[RND];
+#pragma unroll
+        for (int q = 0; q < RND; ++q) {
+          const int item = q * 32 + lane;
+          const int rl = item / IPR;
+          const int c = item - rl * IPR;
+          const int srow = __shfl_sync(0xffffffffu, mine, rl < C::RPW ? rl : 0);
+          raw[q] = make_uint4(0u, 0u, 0u, 0u);
+          sc[q] = 0.0f;
+          if (item < C::RPW * IPR && srow >= 0 && c < CC + RC) {
+            const uint8_t* rp = kv8 + static_cast<int64_t>(srow) * R::ROW_BYTES;
+            if (c < CC) {
+              raw[q] = __ldg(reinterpret_cast<const uint4*>(rp + 16 * c));
+              sc[q] = __ldg(reinterpret_cast<const float*>(rp + R::SCALE_OFF) + (16 * c) / R::TILE);
+            } else {
+              raw[q] = __ldg(reinterpret_cast<const uint4*>(rp + R::ROPE_OFF + 16 * (c - CC)));
+            }
+          }
+        }
+        nxt = row_index(it + 1);
+        if (it == C::NST - 1) ok = mbar_wait_warp(q_moved, 0, abort_flag);
+        if (ok) ok = mbar_wait_warp(&kv_empty[sl], (use & 1u) ^ 1u, abort_flag);
+        if (!ok) break;
+        uint8_t* stage = smem + C::OFF_KV + sl * C::KV_BYTES;
+#pragma unroll
+        for (int q = 0; q < RND; ++q) {
+          const int item = q * 32 + lane;
+          const int rl = item / IPR;
+          const int c = item - rl * IPR;
+          if (item < C::RPW * IPR) {
+            const int r = C::RPW * pw + rl;
+            if (c < CC) {
+              uint4 lo, hi;
+              fp8x16_to_bf16x16(raw[q], sc[q], lo, hi);
+              const int k0 = 2 * c, k1 = 2 * c + 1;  // bf16 chunks of dims 16c .. 16c + 15
+              *reinterpret_cast<uint4*>(stage + (k0 >> 3) * C::ATOM_COL + sw128_offset(r, k0 & 7)) = lo;
+              *reinterpret_cast<uint4*>(stage + (k1 >> 3) * C::ATOM_COL + sw128_offset(r, k1 & 7)) = hi;
+            } else {
+              const int k = c < CC + RC ? DC / 8 + (c - CC) : D / 8 + (c - CC - RC);
+              *reinterpret_cast<uint4*>(stage + (k >> 3) * C::ATOM_COL + sw128_offset(r, k & 7)) = raw[q];
+            }
+          }
+        }
+        fence_proxy_async_smem();  // generic stores -> the tensor cores' reads
+        mbar_arrive(&kv_full[sl]);
+      }
+    } else
     for (int it = 0; it < n_tiles && ok; ++it) {
       const int sl = it % C::NST;
       const uint32_t use = static_cast<uint32_t>(it / C::NST);

@@ -126,6 +126,9 @@ __device__ __forceinline__ bool mbar_wait_cluster_all(uint64_t* bar, uint32_t pa
   return __all_sync(0xffffffffu, ok);
 }
 
+// PAGED: the caches are paged (rows translated through the block table);
+// contiguous calls run without that code in their gather loops.
+template <bool PAGED>
 __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     sparse_mla_pipe_kernel(const __grid_constant__ CUtensorMap kvmap, const __grid_constant__ CUtensorMap qmap,
                            const __grid_constant__ CUtensorMap pmap, const PipeParams p) {
@@ -393,7 +396,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       const bool leader = gl == 0;
       const bool active = gl < 16 * 9;
       const int g = gl / 9, a = gl - (gl / 9) * 9;
-      const int32_t row0 = p.cm.paged() ? 0 : b * p.L_max;  // stand-in row for invalid keys
+      const int32_t row0 = b * p.L_max;  // contiguous: the sequence's first row (the stand-in for invalid keys)
       {
         // stage this split's indices (eight independent loads in flight per thread)
         const int nk = k_end - k_begin;
@@ -438,7 +441,11 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           for (int i = 0; i < 4; ++i) {
             const bool v = cur[i] >= 0 && cur[i] < len;
             if (a == 0 && cur[i] != -1 && !v) set_device_status(DSA_ERR_DEVICE_INDEX);
-            y[i] = v ? p.cm.row_checked(b, cur[i]) : row0;
+            y[i] = row0 + (v ? cur[i] : 0);
+          }
+          if constexpr (PAGED) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[i] = (cur[i] >= 0 && cur[i] < len) ? p.cm.row_checked(b, cur[i]) : 0;
           }
           tma_gather4(smem_u32(smem + C::A_OFF_K + sl * C::K_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0], y[1],
                       y[2], y[3], &kv_full[sl]);
@@ -549,7 +556,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       const bool leader = gl == 0;
       const bool active = gl < 16 * 8;
       const int g = gl >> 3, a = gl & 7;
-      const int32_t row0 = p.cm.paged() ? 0 : b * p.L_max;  // stand-in row for invalid keys
+      const int32_t row0 = b * p.L_max;  // contiguous: the sequence's first row (the stand-in for invalid keys)
       auto load_rows = [&](int tile, int (&y)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -584,9 +591,13 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           if (active) {
             int y[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              bool rok;
-              y[i] = (cur[i] >= 0 && cur[i] < len) ? p.cm.row(b, cur[i], rok) : row0;
+            for (int i = 0; i < 4; ++i) y[i] = row0 + ((cur[i] >= 0 && cur[i] < len) ? cur[i] : 0);
+            if constexpr (PAGED) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                bool rok;
+                y[i] = (cur[i] >= 0 && cur[i] < len) ? p.cm.row(b, cur[i], rok) : 0;
+              }
             }
             tma_gather4(smem_u32(smem + C::B_OFF_V + sl * C::V_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0],
                         y[1], y[2], y[3], &v_full[sl]);

@@ -32,8 +32,12 @@ class DeviceWorkload:
     k_bf16: Optional[torch.Tensor]   # bf16 keys (kept for the FP8 cache write)
     q: torch.Tensor
     kv: torch.Tensor
+    q_mx: Optional[torch.Tensor] = None   # MXFP8 index inputs: E8M0 bytes of q_idx / k_cache
+    k_mx: Optional[torch.Tensor] = None
 
     def indexer_in(self) -> B.dsa_indexer_in:
+        if self.q_mx is not None:
+            return B.indexer_in(self.q_idx, self.w, self.k_cache, q_mx=self.q_mx, k_mx=self.k_mx)
         return B.indexer_in(self.q_idx, self.w, self.k_cache, self.k_scale,
                             self.wl.scale_group if self.k_scale is not None else None)
 
@@ -98,7 +102,8 @@ def to_paged(dw: DeviceWorkload, page_size: int, seed: int = 0, spare_pages: int
 
     Page placement comes from :func:`.workloads.page_layout`; rows are copied
     page by page (layout only). Pool rows no sequence owns hold ``fill`` (FP8
-    codes: 0x7E, scales: 1), so a kernel that read a wrong row would show it.
+    index-key codes: 0x7E, scales: 1; packed FP8 KV rows: bytes 0x11), so a
+    kernel that read a wrong row would show it.
     """
     from . import workloads as W
     wl = dw.wl
@@ -120,10 +125,37 @@ def to_paged(dw: DeviceWorkload, page_size: int, seed: int = 0, spare_pages: int
         pool[have] = flat[src_t[have]]
         return pool
 
-    fp8 = dw.k_scale is not None
+    fp8 = dw.k_scale is not None or dw.k_mx is not None
     k_cache = scatter(dw.k_cache, 0x7E if fp8 else fill)
-    k_scale = scatter(dw.k_scale, 1.0) if fp8 else None
-    kv = scatter(dw.kv, fill)
+    k_scale = scatter(dw.k_scale, 1.0) if dw.k_scale is not None else None
+    k_mx = scatter(dw.k_mx, 127) if dw.k_mx is not None else None   # E8M0 127 = 2^0
+    kv = scatter(dw.kv, 0x11 if dw.kv.dtype == torch.uint8 else fill)  # packed FP8 rows: finite filler
     batch = B.Batch(dw.batch.cu_q, dw.batch.q_pos, dw.batch.seq_lens, wl.Lmax,
                     block_table=torch.from_numpy(table).to(dev), page_size=page_size, num_pages=num_pages)
-    return dataclasses.replace(dw, batch=batch, k_cache=k_cache, k_scale=k_scale, kv=kv, k_bf16=None)
+    return dataclasses.replace(dw, batch=batch, k_cache=k_cache, k_scale=k_scale, kv=kv, k_bf16=None, k_mx=k_mx)
+
+
+def with_fp8_kv(dw: DeviceWorkload) -> DeviceWorkload:
+    """The same workload with its latent KV cache written as packed FP8 rows
+    by the library's own cache-write step (dsa_quantize_kv), as in serving."""
+    wl = dw.wl
+    rows = dw.kv.reshape(-1, wl.D)
+    kv8 = torch.empty((rows.shape[0], B.dsa_kv_fp8_row_bytes(wl.dc, wl.dr)), dtype=torch.uint8, device=dw.kv.device)
+    B.dsa_quantize_kv(rows, wl.dc, kv8)
+    return dataclasses.replace(dw, kv=kv8.reshape(dw.kv.shape[:-1] + (kv8.shape[-1],)))
+
+
+def with_mxfp8_index(dw: DeviceWorkload) -> DeviceWorkload:
+    """The same workload with MXFP8 index queries and keys (group 32, E8M0
+    scales), written by the library's dsa_quantize_mxfp8 from the bf16 ones."""
+    wl = dw.wl
+    dev = dw.q.device
+    keys = dw.k_bf16 if dw.k_bf16 is not None else dw.k_cache
+    assert keys.dtype == torch.bfloat16, "MXFP8 index inputs are made from bf16 keys"
+    k8 = torch.empty(keys.shape, dtype=torch.uint8, device=dev)
+    kmx = torch.empty(keys.shape[:-1] + (wl.dI // 32,), dtype=torch.uint8, device=dev)
+    B.dsa_quantize_mxfp8(keys, k8, kmx)
+    q8 = torch.empty(dw.q_idx.shape, dtype=torch.uint8, device=dev)
+    qmx = torch.empty(dw.q_idx.shape[:-1] + (wl.dI // 32,), dtype=torch.uint8, device=dev)
+    B.dsa_quantize_mxfp8(dw.q_idx, q8, qmx)
+    return dataclasses.replace(dw, q_idx=q8, k_cache=k8, k_scale=None, k_bf16=None, q_mx=qmx, k_mx=kmx)

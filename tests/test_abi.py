@@ -25,7 +25,7 @@ def lib():
 def _declared():
     text = open(os.path.join(ROOT, "include", "dsa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -91,6 +91,16 @@ def test_indexer_validation(lib):
     assert _scores(lib, _batch(), _idx_in(key_dtype=B.DSA_KEY_FP8_E4M3)) == B.DSA_ERR_INVALID_ARGUMENT
     assert _scores(lib, _batch(), _idx_in(key_dtype=B.DSA_KEY_FP8_E4M3, k_scale=FAKE, scale_group=32)) == \
         B.DSA_ERR_UNSUPPORTED_SHAPE
+    # MXFP8: both scale arrays, groups of 32, and a workspace for the widened queries
+    mx = dict(key_dtype=B.DSA_KEY_MXFP8, scale_group=32, q_scale_e8m0=FAKE, k_scale_e8m0=FAKE)
+    assert _scores(lib, _batch(), _idx_in(**dict(mx, k_scale_e8m0=None))) == B.DSA_ERR_INVALID_ARGUMENT
+    assert _scores(lib, _batch(), _idx_in(**dict(mx, scale_group=128))) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert _scores(lib, _batch(), _idx_in(**dict(mx, q_scale_e8m0=MIS))) == B.DSA_ERR_MISALIGNED
+    assert _scores(lib, _batch(), _idx_in(**mx)) == B.DSA_ERR_WORKSPACE_TOO_SMALL
+    assert lib.dsa_quantize_mxfp8(FAKE, 4, 48, FAKE, FAKE, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
+    assert lib.dsa_quantize_mxfp8(FAKE, 4, 64, MIS, FAKE, None) == B.DSA_ERR_MISALIGNED
+    assert lib.dsa_fused_decode_noalloc(ctypes.byref(_batch()), ctypes.byref(_idx_in(**mx)), ctypes.byref(_mla_in()),
+                                        16, FAKE, None, None, None) == B.DSA_ERR_UNSUPPORTED_SHAPE
     assert _scores(lib, _batch(), _idx_in(), scores=None) == B.DSA_ERR_INVALID_ARGUMENT
     assert _scores(lib, _batch(), _idx_in(), ld=100) == B.DSA_ERR_INVALID_ARGUMENT
     assert _scores(lib, _batch(batch=70000, max_seq_len=40000), _idx_in()) == B.DSA_ERR_UNSUPPORTED_SHAPE
@@ -147,11 +157,13 @@ def test_fused_and_quant_validation(lib):
 
 def test_workspace_sizes(lib):
     b = _batch(num_q=32, batch=32, max_seq_len=8192)
-    assert lib.dsa_workspace_size(B.DSA_OP_INDEXER_SCORES, ctypes.byref(b), 2048, 64, 128) == 0
+    # the indexer needs room only for MXFP8 queries widened to bf16 (T x H_I x d_I x 2 bytes)
+    qb = 32 * 64 * 128 * 2
+    assert lib.dsa_workspace_size(B.DSA_OP_INDEXER_SCORES, ctypes.byref(b), 2048, 64, 128) == qb
     assert lib.dsa_workspace_size(B.DSA_OP_TOPK, ctypes.byref(b), 2048, 64, 128) == 0
     fused = lib.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, ctypes.byref(b), 2048, 64, 128)
     mla = lib.dsa_workspace_size(B.DSA_OP_SPARSE_MLA, ctypes.byref(b), 2048, 64, 128)
-    assert fused == 32 * 8192 * 4 + 32 * 2048 * 4 + mla
+    assert fused == 32 * 8192 * 4 + 32 * 2048 * 4 + mla + qb
     assert lib.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, None, 2048, 64, 128) == 0
 
 

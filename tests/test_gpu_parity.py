@@ -114,6 +114,24 @@ def test_indexer_decode_shapes_integer_exact(HI, dI, key_dtype):
         assert np.all(got[t, nv[t]:(nv[t] + 127) // 128 * 128] == -np.inf)
 
 
+@pytest.mark.parametrize("Lmax", [1001, 1000])
+def test_indexer_decode_fp8_scale_rows(Lmax):
+    """FP8 decode: with max_seq_len a multiple of 4 every tile's 128 scales
+    are copied into its stage (the last tile of the cache clipped at the end);
+    otherwise each key's scale is read from global memory. Integer values:
+    scores exact either way."""
+    lens = (Lmax, 130, 1, Lmax - 3)
+    wl = W.scaled("c5i", B=4, Lmax=Lmax, lens=lens, T_per_seq=1, K=64, HI=64, dI=128, key_dtype="fp8",
+                  integer=True)
+    dw = DV.to_device(wl)
+    codes, scales = oracle_codes(dw)
+    got = _np(gpu_scores(dw))
+    want = oracle.indexer_scores(wl, k_codes=codes, k_scales=scales)
+    nv = wl.n_valid()
+    for t in range(wl.T):
+        assert np.array_equal(got[t, :nv[t]], want[t, :nv[t]].astype(np.float32)), t
+
+
 @pytest.mark.parametrize("key_dtype", ["bf16", "fp8"])
 def test_indexer_decode_ranges_span_many_tokens(key_dtype):
     """200 short sequences (one of them empty): the flattened key-tile list has
