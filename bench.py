@@ -57,6 +57,9 @@ WORKLOAD_TEXT = {
 # with MXFP8 index queries and keys.
 FP8_KV = {"c2kv8": "c2"}
 MX_INDEX = {"c3mx": "c3"}
+# Ragged batches whose sequences are split across ranks (longest first, no
+# exchange: sequences are independent); the others run one copy per rank.
+SHARDED = ("c3",)
 
 
 def _peaks():
@@ -248,13 +251,21 @@ class Runner:
     """One workload resident on the device in rotating copies, run through
     dsa_fused_decode (the whole chain as one C-ABI call per step)."""
 
-    def __init__(self, name, dev, copies):
+    def __init__(self, name, dev, copies, rank=0, world=1):
         import torch
         from indexed_sparse_attention_relu_b200 import binding as B
         from indexed_sparse_attention_relu_b200 import device as DV
         from indexed_sparse_attention_relu_b200 import workloads as W
         self.B = B
-        self.wl = wl = W.make(FP8_KV.get(name, MX_INDEX.get(name, name)), with_caches=False)
+        wl = W.make(FP8_KV.get(name, MX_INDEX.get(name, name)), with_caches=False)
+        # tokens each rank processes per step (one full copy per rank unless sharded)
+        self.units = [wl.T] * world
+        if world > 1 and name in SHARDED:
+            from indexed_sparse_attention_relu_b200 import multi
+            shards = multi.shard_sequences(wl.seq_lens, world)
+            self.units = [int(sum(wl.cu_q[b + 1] - wl.cu_q[b] for b in sh)) for sh in shards]
+            wl = W.select_sequences(wl, shards[rank])
+        self.wl = wl
         self.dev = dev
         base = DV.to_device(wl, dev, keep_bf16_keys=name in MX_INDEX)
         self.kv_row_bytes = None
@@ -493,7 +504,8 @@ def main():
     build_mod.build()
     B.load()
 
-    run = Runner(args.config, dev, args.copies)
+    run = Runner(args.config, dev, args.copies, rank=rank, world=world)
+    sharded = world > 1 and args.config in SHARDED
     wl = run.wl
     T, K = wl.T, wl.K
     stream = torch.cuda.current_stream(dev)
@@ -503,7 +515,7 @@ def main():
     # the job's time is its slowest rank's; every rank ran its own T queries
     total_ms = multi.max_over_ranks(total_ms, dist if world > 1 else None, dev)
     ms_per_step = total_ms / args.steps
-    value = multi.job_throughput([T] * world, ms_per_step)
+    value = multi.job_throughput(run.units, ms_per_step)
 
     e2e_ms, h2d, d2h = e2e_pipelined(run, args.steps, args.warmup, dev)
     e2e_ms = multi.max_over_ranks(e2e_ms, dist if world > 1 else None, dev)
@@ -538,11 +550,14 @@ def main():
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.config], "name": args.config, "B": wl.B, "L_max": wl.Lmax,
                    "T": T, "K": K, "H_I": wl.HI, "d_I": wl.dI, "H": wl.H, "d_c": wl.dc, "d_rope": wl.dr,
-                   "index_keys": wl.key_dtype, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "index_keys": wl.key_dtype,
+                   "parallelism": (f"sequences sharded x{world} (longest first)" if sharded else f"replicas x{world}")
+                   if world > 1 else "single GPU",
                    "l2": f"{len(run.copies)} rotating input copies ({run.resident_bytes / 1e9:.2f} GB) > 126 MB L2"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
@@ -553,7 +568,7 @@ def main():
         "stage_ms": stage_ms,
         "stage_ms_note": "second K-step pass, eager launches with CUDA events between the stages",
         "clocks": clocks,
-        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": sum(run.units) / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "note": "pinned host buffers; uploads and downloads on their own streams, double buffered"},
         "gpu_launches": launches_per_step * args.steps,
@@ -567,6 +582,13 @@ def main():
         line["cpu_baseline"] = {"value": n / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
                                 "sample": f"{min(args.cpu_tokens, wl.T)} query tokens of the same workload (full "
                                           f"causal history), fp64, repeated to {n} tokens in {dt:.1f} s"}
+        # the same oracle on one core (OpenMP threads = 1), a shorter sample
+        import oracle
+        oracle.set_num_threads(1)
+        n1, dt1, _ = run_cpu_oracle(wl, 1, min_seconds=min(args.cpu_seconds, 3.0))
+        oracle.set_num_threads(thr)
+        line["cpu_baseline"]["single_core"] = {"value": n1 / dt1, "unit": UNIT, "cores": 1,
+                                               "sample": f"1 query token, repeated to {n1} in {dt1:.1f} s"}
     if world == 1 and args.extra:
         line["configs"] = []
         for name in [x for x in args.extra.split(",") if x and x != args.config]:

@@ -163,6 +163,7 @@ class Workload:
     seed: int
     integer_valued: bool
     laws: dict = dataclasses.field(default_factory=dict, repr=False)  # cache tag -> value law
+    seq_ids: Optional[np.ndarray] = None  # sequences of a parent workload these are (select_sequences)
 
     @property
     def D(self) -> int:
@@ -181,7 +182,8 @@ class Workload:
         """Cache rows [seq_len_b, dim] of sequence b (tag 'k_idx' or 'kv'), regenerated
         from the same counter-based streams the full cache is drawn from."""
         dim = self.dI if tag == "k_idx" else self.D
-        return _draw_rows(self.seed, f"{tag}/{b}", int(self.seq_lens[b]), dim, self.laws[tag], round_bf16=True)
+        src = b if self.seq_ids is None else int(self.seq_ids[b])
+        return _draw_rows(self.seed, f"{tag}/{src}", int(self.seq_lens[b]), dim, self.laws[tag], round_bf16=True)
 
 
 def _cache(seed, tag, B, Lmax, lens, dim, law, rows_needed=None):
@@ -363,6 +365,23 @@ def restrict(wl: Workload, rows) -> Workload:
     return dataclasses.replace(wl, B=len(seqs), T=len(rows), Lmax=Lmax, cu_q=cu, q_pos=wl.q_pos[rows].copy(),
                                seq_lens=lens, q_idx=wl.q_idx[rows].copy(), w=wl.w[rows].copy(),
                                q=wl.q[rows].copy(), k_idx=k_idx, kv=kv), rows
+
+
+def select_sequences(wl: Workload, seqs) -> Workload:
+    """The sequences ``seqs`` (ascending) of a workload made without host caches,
+    with all their query tokens: the share of one rank when a batch of
+    independent sequences is split across GPUs. Cache rows are regenerated
+    from the parent's streams (seq_ids), so values are identical."""
+    seqs = np.asarray(sorted(int(b) for b in seqs), np.int64)
+    assert wl.k_idx is None and wl.kv is None, "select_sequences works on workloads made without host caches"
+    b_of = wl.seq_of_token()
+    rows = np.nonzero(np.isin(b_of, seqs))[0]
+    counts = np.array([int(wl.cu_q[b + 1] - wl.cu_q[b]) for b in seqs], np.int64)
+    cu = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    parent = wl.seq_ids if wl.seq_ids is not None else np.arange(wl.B)
+    return dataclasses.replace(wl, B=len(seqs), T=len(rows), cu_q=cu, q_pos=wl.q_pos[rows].copy(),
+                               seq_lens=wl.seq_lens[seqs].astype(np.int32), q_idx=wl.q_idx[rows].copy(),
+                               w=wl.w[rows].copy(), q=wl.q[rows].copy(), seq_ids=parent[seqs].copy())
 
 
 CONFIGS = tuple(_SEEDS)

@@ -168,15 +168,16 @@ void oracle_indexer_scores(int32_t B, int32_t Lmax, const int32_t *cu_q, const i
                            const uint8_t *k_fp8, const float *k_scale, int32_t group,
                            int32_t n_rows, const int32_t *rows, double *scores, int64_t ld)
 {
-#pragma omp parallel for schedule(dynamic, 1)
+    /* every (row, position) is independent: spread them over the threads */
+#pragma omp parallel for collapse(2) schedule(dynamic, 256)
     for (int32_t r = 0; r < n_rows; ++r) {
-        int32_t t = rows[r];
-        int32_t b = seq_of_token(cu_q, B, t);
-        int32_t nv = q_pos[t] + 1;
-        if (nv > seq_lens[b])
-            nv = seq_lens[b];
-        double *out = scores + (int64_t)r * ld;
         for (int32_t s = 0; s < Lmax; ++s) {
+            int32_t t = rows[r];
+            int32_t b = seq_of_token(cu_q, B, t);
+            int32_t nv = q_pos[t] + 1;
+            if (nv > seq_lens[b])
+                nv = seq_lens[b];
+            double *out = scores + (int64_t)r * ld;
             if (s >= nv) {
                 out[s] = -INFINITY;
                 continue;

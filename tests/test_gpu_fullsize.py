@@ -67,8 +67,9 @@ def _run(name, extra_rows, seed, rank_in_fp32=False):
 
 
 def test_c2_decode_full():
-    """32 x 8192 decode, BF16 index keys: the benchmark's workload and launch."""
-    _run("c2", extra_rows=6, seed=2)
+    """32 x 8192 decode, BF16 index keys: the benchmark's workload and launch;
+    every one of its 32 query rows is checked."""
+    _run("c2", extra_rows=32, seed=2)
 
 
 def test_c3_ragged_fp8_full():

@@ -207,3 +207,22 @@ def test_zigzag_context_parallel_prefill_two_gloo_ranks():
     for _, idx_parts, out_parts in got:           # every rank holds the whole result
         assert np.array_equal(multi.zigzag_restore(idx_parts, wl.T, world), want_idx)
         assert np.array_equal(multi.zigzag_restore(out_parts, wl.T, world), want_out)
+
+
+def test_sharded_ragged_decode_covers_every_token_once():
+    """bench.py --gpus N on the ragged decode gives each rank whole sequences
+    (longest first, no exchange): every query token lands on exactly one rank,
+    the per-rank workloads regenerate the same cache rows as the full batch,
+    and the loads are balanced to within the longest sequence."""
+    wl = W.make("c3", with_caches=False)
+    for world in (2, 3, 8):
+        shards = multi.shard_sequences(wl.seq_lens, world)
+        parts = [W.select_sequences(wl, sh) for sh in shards]
+        assert sum(p.T for p in parts) == wl.T
+        seen = np.concatenate([p.seq_ids for p in parts])
+        assert sorted(seen.tolist()) == list(range(wl.B))
+        loads = [int(p.seq_lens.sum()) for p in parts]
+        assert max(loads) - min(loads) <= int(wl.seq_lens.max())
+    p = W.select_sequences(wl, [5, 17])
+    assert np.array_equal(p.seq_rows("k_idx", 1), wl.seq_rows("k_idx", 17))
+    assert np.array_equal(p.q_pos, wl.q_pos[[5, 17]])
