@@ -5,13 +5,14 @@ Default workload: decode, batch 32 x 8192 context, one new token each
 (H_I=64, d_I=128, K=2048, 128 MLA heads, 512+64 latent dims, BF16), timed as
 one ``dsa_fused_decode`` call per step through the C ABI. Prints one JSON line.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c3|c4|c5] [--extra c3,c3mx,c2kv8,c4,c5]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c3|c4|c5] [--extra c3,c3mx,c2kv8,c2pg,c4,c5]
   python bench.py --impl reference ...     # the CPU oracle, timed on host cores
 
 The JSON line's headline is the decode workload; ``configs`` adds one block
-per extra workload (the ragged decode with FP8 or MXFP8 index inputs and the
-decode over an FP8 latent KV cache against the HBM roofline, the prefills
-against the dense tensor-core peak), each graph-timed the same way.
+per extra workload (the ragged decode with FP8 or MXFP8 index inputs, the
+decode over an FP8 latent KV cache or over paged caches against the HBM
+roofline, the prefills against the dense tensor-core peak), each graph-timed
+the same way.
 
 Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
 device synchronize, timed with CUDA events on the launch stream; max over
@@ -48,6 +49,8 @@ WORKLOAD_TEXT = {
     "c5": "chunked prefill: 4 x (131072 prefix + 8192 chunk); FP8 index keys; K=2048; 128 MLA heads",
     "c3mx": "ragged decode: batch 64, context U[1024,65536]; MXFP8 index queries and keys (E4M3, one E8M0 "
             "scale per 32 elements); K=2048; 128 MLA heads, 576-dim BF16 latent rows",
+    "c2pg": "decode: batch 32 x 8192 context, 1 query each; H_I=64 d_I=128 BF16; K=2048; 128 MLA heads; "
+            "paged caches (64-row pages in a shuffled pool, one block table)",
     "c2kv8": "decode: batch 32 x 8192 context, 1 query each; H_I=64 d_I=128 BF16 index keys; K=2048; "
              "128 MLA heads; FP8 latent KV cache (4 x 128-element tiles per token, fp32 scales, rope BF16: "
              "656-byte rows)",
@@ -57,6 +60,7 @@ WORKLOAD_TEXT = {
 # with MXFP8 index queries and keys.
 FP8_KV = {"c2kv8": "c2"}
 MX_INDEX = {"c3mx": "c3"}
+PAGED = {"c2pg": "c2"}  # every cache in a pool of 64-row pages under a block table
 # Ragged batches whose sequences are split across ranks (longest first, no
 # exchange: sequences are independent); the others run one copy per rank.
 SHARDED = ("c3",)
@@ -257,7 +261,7 @@ class Runner:
         from indexed_sparse_attention_relu_b200 import device as DV
         from indexed_sparse_attention_relu_b200 import workloads as W
         self.B = B
-        wl = W.make(FP8_KV.get(name, MX_INDEX.get(name, name)), with_caches=False)
+        wl = W.make(FP8_KV.get(name, MX_INDEX.get(name, PAGED.get(name, name))), with_caches=False)
         # tokens each rank processes per step (one full copy per rank unless sharded)
         self.units = [wl.T] * world
         if world > 1 and name in SHARDED:
@@ -273,6 +277,8 @@ class Runner:
         if name in MX_INDEX:  # the library's MXFP8 quantisation of q_I and k_I, outside the timed region
             base = DV.with_mxfp8_index(base)
             self.key_row_bytes = wl.dI + wl.dI // 32
+        if name in PAGED:
+            base = DV.to_paged(base, 64, seed=wl.seed)
         if name in FP8_KV:  # the library's FP8 KV cache write, outside the timed region
             base = DV.with_fp8_kv(base)
             self.kv_row_bytes = B.dsa_kv_fp8_row_bytes(wl.dc, wl.dr)
@@ -425,7 +431,7 @@ def extra_block(name, args, dev, stream):
     """One graph-timed measurement of another workload, with its roofline."""
     import torch
     t0 = time.time()
-    decode = name in ("c3", "c3mx", "c2kv8")
+    decode = name in ("c3", "c3mx", "c2kv8", "c2pg")
     steps = args.extra_steps_decode if decode else args.extra_steps_prefill
     run = Runner(name, dev, copies=2)
     wl = run.wl
@@ -474,7 +480,7 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=1, help="query tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one CUDA graph")
-    ap.add_argument("--extra", default="c3,c3mx,c2kv8,c4,c5",
+    ap.add_argument("--extra", default="c3,c3mx,c2kv8,c2pg,c4,c5",
                     help="comma-separated extra workloads measured after the headline (single GPU only; '' for none)")
     ap.add_argument("--extra-steps-decode", type=int, default=20)
     ap.add_argument("--extra-steps-prefill", type=int, default=3)
