@@ -46,8 +46,12 @@
  *      MLA (d_latent, d_rope): (512, 64), (64, 16)
  *      MLA heads H: 1..64, or 128
  *      top-K k: 1..2048
- *    FP8 index keys need scale_group == d_I (one scale per key).
- *  - Alignment: every tensor pointer must be 16-byte aligned.
+ *      paged caches: page_size a positive multiple of 64
+ *    FP8 index keys need scale_group == d_I (one scale per key); MXFP8 index
+ *    inputs need scale_group == 32. FP8 latent KV rows come in the packed
+ *    layout of dsa_quantize_kv for either MLA shape.
+ *  - Alignment: every tensor pointer must be 16-byte aligned (the block table:
+ *    4-byte aligned).
  */
 #ifndef DSA_H_
 #define DSA_H_

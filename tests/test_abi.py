@@ -222,3 +222,14 @@ def test_header_supported_shapes_match_validation(lib):
         assert lib.dsa_topk(ctypes.byref(empty), FAKE, 256, k, FAKE, None, 0, None) == want, k
         got = lib.dsa_sparse_mla_attn(ctypes.byref(empty), ctypes.byref(_mla_in()), FAKE, k, FAKE, None, None, 0, None)
         assert got == want, k
+
+
+def test_header_page_size_rule_matches_validation(lib):
+    """The header's paged-cache line (a positive multiple of N) against validation."""
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    mult = int(re.search(r"paged caches: page_size a positive multiple of (\d+)", text).group(1))
+    assert mult == 64
+    for ps in (32, 64, 96, 128, 192, 256, 1000, 1024):
+        want = B.DSA_OK if ps % mult == 0 else B.DSA_ERR_UNSUPPORTED_SHAPE
+        b = _batch(num_q=0, block_table=FAKE, page_size=ps, num_pages=4)
+        assert _scores(lib, b, _idx_in()) == want, ps
