@@ -52,6 +52,13 @@
  *    layout of dsa_quantize_kv for either MLA shape.
  *  - Alignment: every tensor pointer must be 16-byte aligned (the block table:
  *    4-byte aligned).
+ *  - Debug build (libdsa_debug.so, compiled with DSA_DEBUG): before the
+ *    attention gathers any row, the host checks every index (the call then
+ *    synchronises its stream) and returns DSA_ERR_INVALID_ARGUMENT naming the
+ *    first one that is neither -1 nor inside its sequence; the tensor-core
+ *    kernels guard the end of their shared-memory layout with a canary and
+ *    report DSA_ERR_DEVICE_LAYOUT if it was overwritten. Calls of the debug
+ *    build cannot be captured in a CUDA graph.
  */
 #ifndef DSA_H_
 #define DSA_H_

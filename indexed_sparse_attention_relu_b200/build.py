@@ -1,6 +1,6 @@
 """Builds libdsa.so (the C-ABI CUDA library) in-tree with nvcc for sm_100a.
 
-Usage: python -m indexed_sparse_attention_relu_b200.build [--force] [--verbose]
+Usage: python -m indexed_sparse_attention_relu_b200.build [--force] [--verbose] [--debug]
 """
 from __future__ import annotations
 
@@ -36,19 +36,29 @@ def _sources():
                   + [os.path.join(ROOT, "include", "dsa.h")])
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+DEBUG_LIB = os.path.join(PKG, "libdsa_debug.so")
+
+
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/dsa.cu into libdsa.so unless it is up to date."""
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), os.path.join(CSRC, "dsa.cu"), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile csrc/dsa.cu into libdsa.so unless it is up to date.
+
+    debug=True builds libdsa_debug.so with DSA_DEBUG defined: every gathered
+    row index is checked on the host before the attention runs (the calls
+    then synchronise), and the tensor-core kernels guard the end of their
+    shared memory with a canary that reports DSA_ERR_DEVICE_LAYOUT."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DDSA_DEBUG"] if debug else []), "-I", os.path.join(ROOT, "include"),
+           os.path.join(CSRC, "dsa.cu"), "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,9 +66,15 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose", action="store_true")
+    ap.add_argument("--debug", action="store_true", help="build libdsa_debug.so (DSA_DEBUG)")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.verbose, debug=a.debug))

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "dsa_common.cuh"
 #include "indexer.cuh"
@@ -293,7 +294,38 @@ size_t mla_ws_bytes(const dsa_batch* bt, int k) {
   return bp > need ? bp : need;
 }
 
+// ---------------------------------------------------------------- debug build
+#ifdef DSA_DEBUG
+// Host check of every index the attention is about to gather: copies the
+// indices and the batch metadata to the host (synchronising the stream) and
+// requires each to be -1 or a position inside its sequence.
+dsa_status debug_check_indices(const dsa_batch* bt, const int32_t* idx, int k, cudaStream_t st) {
+  const int T = bt->num_q, B = bt->batch;
+  std::vector<int32_t> h_idx(static_cast<size_t>(T) * k), cu(B + 1), lens(B);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(h_idx.data(), idx, h_idx.size() * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(cu.data(), bt->cu_q, cu.size() * 4, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(lens.data(), bt->seq_lens, lens.size() * 4, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "DSA_DEBUG index check: %s", cudaGetErrorString(e));
+  int b = 0;
+  for (int t = 0; t < T; ++t) {
+    while (b + 1 < B && cu[b + 1] <= t) ++b;
+    const int len = lens[b] < bt->max_seq_len ? lens[b] : bt->max_seq_len;
+    for (int i = 0; i < k; ++i) {
+      const int v = h_idx[static_cast<size_t>(t) * k + i];
+      if (v != -1 && (v < 0 || v >= len))
+        return fail(DSA_ERR_INVALID_ARGUMENT, "DSA_DEBUG: idx[%d][%d] = %d outside [-1, %d)", t, i, v, len);
+    }
+  }
+  return DSA_OK;
+}
+#endif
+
 // ---------------------------------------------------------------- launches
+// Dynamic shared memory of a tensor-core kernel: its layout, plus (DSA_DEBUG)
+// the canary after it.
+int smem_request(int layout_bytes) { return kCanaryBytes ? canary_offset(layout_bytes) + kCanaryBytes : layout_bytes; }
+
 template <typename Kern>
 dsa_status set_smem(Kern k, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -322,7 +354,7 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   dsa_status s = make_key_map(&map, in->k_cache, cache_rows(bt), DIN, FP8, key_box_rows(bt));
   if (s != DSA_OK) return s;
   auto kern = indexer_scores_kernel<HI, DIN, G, KF>;
-  if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
+  if ((s = set_smem(kern, smem_request(C::SMEM_BYTES))) != DSA_OK) return s;
   const int sms = num_sms();
   const int64_t groups64 = static_cast<int64_t>((bt->num_q + G - 1) / G) + bt->batch;
   const int groups = static_cast<int>(groups64 < bt->num_q ? groups64 : bt->num_q);
@@ -361,7 +393,7 @@ dsa_status launch_indexer_t(const dsa_batch* bt, const dsa_indexer_in* in, float
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(groups, gy);
   cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem_request(C::SMEM_BYTES);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -385,7 +417,7 @@ dsa_status launch_indexer_decode(const dsa_batch* bt, const dsa_indexer_in* in, 
   if (s != DSA_OK) return s;
   if ((s = make_bf16_rows_map(&qmap, in->q, static_cast<int64_t>(bt->num_q) * HI, DIN, HI)) != DSA_OK) return s;
   auto kern = indexer_decode_kernel<HI, DIN, KF>;
-  if ((s = set_smem(kern, C::SMEM_BYTES)) != DSA_OK) return s;
+  if ((s = set_smem(kern, smem_request(C::SMEM_BYTES))) != DSA_OK) return s;
   IdxDecParams p;
   p.cu_q = bt->cu_q;
   p.q_pos = bt->q_pos;
@@ -406,7 +438,7 @@ dsa_status launch_indexer_decode(const dsa_batch* bt, const dsa_indexer_in* in, 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms());
   cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem_request(C::SMEM_BYTES);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -537,7 +569,7 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
                         float* lse, void* ws, size_t ws_bytes, cudaStream_t st, const MlaPlan& pl, bool pdl) {
   using C = MlaCfg<D, DC>;
   auto kern = sparse_mla_kernel<D, DC, FP8KV>;
-  dsa_status s = set_smem(kern, C::SMEM_BYTES);
+  dsa_status s = set_smem(kern, smem_request(C::SMEM_BYTES));
   if (s != DSA_OK) return s;
   const int T = bt->num_q, H = in->n_heads;
   CUtensorMap qmap;
@@ -572,7 +604,7 @@ dsa_status launch_mla_t(const dsa_batch* bt, const dsa_mla_in* in, const int32_t
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(T, hb, pl.splits);
   cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem_request(C::SMEM_BYTES);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -604,11 +636,11 @@ int pipe_max_clusters(int size, int fallback) {
     int n = 0;
     // (no error message is recorded here: a size query may run without a device)
     if (cudaFuncSetAttribute(sparse_mla_pipe_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             PipeCfg::SMEM_BYTES) == cudaSuccess) {
+                             smem_request(PipeCfg::SMEM_BYTES)) == cudaSuccess) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(size, 1, 1);
       cfg.blockDim = dim3(PipeCfg::THREADS);
-      cfg.dynamicSmemBytes = PipeCfg::SMEM_BYTES;
+      cfg.dynamicSmemBytes = smem_request(PipeCfg::SMEM_BYTES);
       cudaLaunchAttribute attr;
       attr.id = cudaLaunchAttributeClusterDimension;
       attr.val.clusterDim.x = size;
@@ -628,7 +660,7 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
                            float* lse, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl) {
   using C = PipeCfg;
   auto kern = bt->block_table ? sparse_mla_pipe_kernel<true> : sparse_mla_pipe_kernel<false>;
-  dsa_status s = set_smem(kern, C::SMEM_BYTES);
+  dsa_status s = set_smem(kern, smem_request(C::SMEM_BYTES));
   if (s != DSA_OK) return s;
   const int T = bt->num_q;
   const MlaPlan pl = pipe_plan(T, k, num_sms());
@@ -686,7 +718,7 @@ dsa_status launch_mla_pipe(const dsa_batch* bt, const dsa_mla_in* in, const int3
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pl.splits, T, 1);
   cfg.blockDim = dim3(C::THREADS);
-  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.dynamicSmemBytes = smem_request(C::SMEM_BYTES);
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   int na = 0;
@@ -812,6 +844,9 @@ dsa_status dsa_sparse_mla_attn(const dsa_batch* batch, const dsa_mla_in* in, con
   if (!aligned16(out) || !aligned16(idx)) return fail(DSA_ERR_MISALIGNED, "idx and out must be 16-byte aligned");
   if (k < 1 || k > 2048) return fail(DSA_ERR_UNSUPPORTED_SHAPE, "k=%d outside [1, 2048]", k);
   if (batch->num_q == 0) return DSA_OK;
+#ifdef DSA_DEBUG
+  if ((s = debug_check_indices(batch, idx, k, reinterpret_cast<cudaStream_t>(stream))) != DSA_OK) return s;
+#endif
   return launch_mla(batch, in, idx, k, out, lse, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -854,6 +889,9 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
     return s;
   if ((s = rec(1)) != DSA_OK) return s;
   if ((s = launch_topk(batch, scores, batch->max_seq_len, k, idx, st, pdl)) != DSA_OK) return s;
+#ifdef DSA_DEBUG
+  if ((s = debug_check_indices(batch, idx, k, st)) != DSA_OK) return s;
+#endif
   if ((s = rec(2)) != DSA_OK) return s;
   if ((s = launch_mla(batch, mla_in, idx, k, out, lse, static_cast<uint8_t*>(ws) + sc_bytes + id_bytes, mla_bytes, st,
                       pdl)) != DSA_OK)

@@ -40,6 +40,39 @@ __device__ uint64_t g_wait_limit_ns = kDefaultWaitLimitNs;
 // (set by dsa_debug_withhold_signal(); 0 in normal operation).
 __device__ int g_debug_withhold = 0;
 
+// ---------------------------------------------------------------- debug build
+// With DSA_DEBUG the tensor-core kernels request kCanaryBytes more dynamic
+// shared memory and thread 0 writes a fixed pattern right after the kernel's
+// layout at entry and checks it at exit: a layout that wrote past its end
+// shows up as DSA_ERR_DEVICE_LAYOUT. Without DSA_DEBUG both are no-ops.
+#ifdef DSA_DEBUG
+constexpr int kCanaryBytes = 16;
+#else
+constexpr int kCanaryBytes = 0;
+#endif
+constexpr int canary_offset(int layout_bytes) { return (layout_bytes + 15) / 16 * 16; }
+__device__ __forceinline__ void canary_set(uint8_t* smem, int layout_bytes) {
+#ifdef DSA_DEBUG
+  if (threadIdx.x == 0)
+    *reinterpret_cast<uint4*>(smem + canary_offset(layout_bytes)) = make_uint4(0xD5A0C0DEu, 0x5EA1ED00u, 0xC0FFEE11u, 0xB200B200u);
+#else
+  (void)smem;
+  (void)layout_bytes;
+#endif
+}
+__device__ __forceinline__ void canary_check(const uint8_t* smem, int layout_bytes) {
+#ifdef DSA_DEBUG
+  if (threadIdx.x == 0) {
+    const uint4 c = *reinterpret_cast<const uint4*>(smem + canary_offset(layout_bytes));
+    if (c.x != 0xD5A0C0DEu || c.y != 0x5EA1ED00u || c.z != 0xC0FFEE11u || c.w != 0xB200B200u)
+      set_device_status(DSA_ERR_DEVICE_LAYOUT);
+  }
+#else
+  (void)smem;
+  (void)layout_bytes;
+#endif
+}
+
 // ---------------------------------------------------------------- cache rows
 // Where logical row s of sequence b lives in a cache (index keys, their FP8
 // scales and the latent KV rows all share it). Contiguous caches: row

@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
     if (threadIdx.x == 0) set_device_status(DSA_ERR_DEVICE_LAYOUT);
     return;
   }
+  canary_set(smem, C::SMEM_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* full = bars;                      // [ST]  TMA -> MMA / converters
   uint64_t* empty = bars + C::ST;             // [ST]  MMA / converters -> TMA
@@ -541,6 +542,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  canary_check(smem, C::SMEM_BYTES);
   // Under programmatic dependent launch this grid may start while the
   // previous kernel of the stream (the attention of the previous call) still
   // runs. It reads nothing that kernel writes, but it must not complete

@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     if (threadIdx.x == 0) set_device_status(DSA_ERR_DEVICE_LAYOUT);
     return;
   }
+  canary_set(smem, C::SMEM_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bars;             // [NST] gather producers -> MMA
   uint64_t* kv_empty = bars + C::NST;   // [NST] MMA (PV done) -> gather producers
@@ -749,6 +750,7 @@ __global__ void __launch_bounds__(MlaCfg<D, DC>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+  canary_check(smem, C::SMEM_BYTES);
 }
 
 }  // namespace dsa

@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     if (threadIdx.x == 0) set_device_status(DSA_ERR_DEVICE_LAYOUT);
     return;
   }
+  canary_set(smem, C::SMEM_BYTES);
   const uint32_t crank = cluster_ctarank();
   const bool score_cta = (crank & 1u) == 0;
   const int split = static_cast<int>(crank >> 1);
@@ -824,6 +825,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+  canary_check(smem, C::SMEM_BYTES);
 }
 
 }  // namespace dsa

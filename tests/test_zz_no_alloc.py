@@ -160,3 +160,29 @@ def test_noalloc_scratch_filled_to_its_last_byte():
     r = B.load().dsa_fused_decode_noalloc(ctypes.byref(bt), ctypes.byref(dw.indexer_in()), ctypes.byref(dw.mla_in()),
                                           K, 0x10000, None, None, None)
     assert r == B.DSA_ERR_WORKSPACE_TOO_SMALL
+
+
+@pytest.mark.gpu
+def test_noalloc_paged_caches_and_fp8_kv():
+    """Paged caches (64-row pages under one block table) with an FP8 latent KV
+    cache: the allocation-free call matches the workspace entry point on the
+    same inputs (indices identical; the attention runs unsplit here)."""
+    from indexed_sparse_attention_relu_b200 import device as DV
+    from indexed_sparse_attention_relu_b200 import workloads as W
+
+    B.load()
+    wl = W.scaled("c2", B=3, Lmax=2600, lens=(2600, 2049, 900), T_per_seq=1, K=1024)
+    dw = DV.to_paged(DV.with_fp8_kv(DV.to_device(wl, "cuda")), 64, seed=5)
+    T, K = wl.T, wl.K
+    nbytes = B.dsa_workspace_size(B.DSA_OP_FUSED_DECODE, dw.batch, K)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out_ref = torch.empty((T, wl.H, wl.dc), dtype=torch.bfloat16, device="cuda")
+    idx_ref = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    B.dsa_fused_decode(dw.batch, dw.indexer_in(), dw.mla_in(), K, out_ref, None, idx_ref, ws, nbytes)
+    torch.cuda.synchronize()
+    ref = out_ref.float().cpu().numpy().astype(np.float64)
+    for call in range(2):
+        out, _, idx = _noalloc_run(dw, K, with_idx_out=True)
+        assert torch.equal(idx, idx_ref), call
+        d = out.float().cpu().numpy().astype(np.float64) - ref
+        assert float(np.abs(d).max()) <= MAX_ABS and float(np.linalg.norm(d) / np.linalg.norm(ref)) <= REL_L2, call
