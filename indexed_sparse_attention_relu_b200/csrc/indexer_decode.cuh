@@ -58,7 +58,7 @@ template <int HI, int DIN, int KF>
 struct IdxDecCfg {
   static constexpr bool FP8 = KF != KF_BF16;             // 8-bit codes, widened by converter warps
   static constexpr int SROW = KF == KF_FP8 ? 4 : KF == KF_MX ? DIN / 32 : 0;  // scale bytes per key row
-  static constexpr int EPI_G = KF == KF_FP8 ? 2 : 1;
+  static constexpr int EPI_G = KF != KF_BF16 ? 2 : 1;
   static constexpr int CONV_W = KF == KF_FP8 ? 6 : KF == KF_MX ? 8 : 0;
   static constexpr int DK = DIN < 64 ? 64 : DIN;         // K padded to whole 128-byte atoms
   static constexpr int AK = DK / 64;                     // atom columns along K
@@ -74,11 +74,11 @@ struct IdxDecCfg {
   static constexpr int Q_TX = AK * HI * 128;             // bytes the query TMA writes per buffer
   static constexpr int W_BYTES = ((HI * 4 + 15) / 16) * 16;
   static constexpr int MAXSEG = 256;                     // segments a CTA can hold (tokens <= MAXSEG)
-  // Epilogue groups of four warps: with FP8 keys two groups, group g taking
+  // Epilogue groups of four warps: with 8-bit keys two groups, group g taking
   // the tiles with it % 2 == g (accumulator g), so two tiles' epilogues run at
-  // once (measured 6 % faster on a ragged FP8 decode). BF16 keys keep one
-  // group; MXFP8 keys, whose widening also applies the block scales, keep one
-  // group and eight converter warps.
+  // once (measured 6 % faster on a ragged FP8 decode, 1 % with MXFP8 keys,
+  // whose widening also applies the block scales and keeps eight converter
+  // warps); BF16 keys keep one group.
   static constexpr int EPI_GROUPS = EPI_G;
   static constexpr int EPI_WARPS = 4 * EPI_GROUPS;
   static constexpr int CONV_WARPS = CONV_W;              // 8-bit -> bf16 converters

@@ -249,6 +249,28 @@ def test_topk_register_rows_full_and_ragged():
     assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
 
 
+@pytest.mark.parametrize("L", [8192, 16384, 32768, 65536])
+def test_topk_threshold_ties_at_each_kernel_limit(L):
+    """Rows of 8192 and 16384 positions (held in registers) and of 32768 and
+    65536 (position bitmaps and a candidate list in shared memory), each at
+    the longest row of its kernel: an all-equal row, integer scores and a few
+    large values over a constant bulk put long runs of ties at the threshold,
+    across thread and chunk boundaries; a shorter row and one of fewer than K
+    positions ride along in the same launch."""
+    rng = np.random.default_rng(L)
+    bulk = np.full(L, 0.5, np.float32)
+    bulk[rng.choice(L, 1500, replace=False)] = 3.0
+    rows = [np.zeros(L, np.float32),
+            np.float32(rng.integers(-4, 5, L)),
+            bulk,
+            W.bf16_round(rng.standard_normal(L).astype(np.float32) * 8),
+            W.bf16_round(rng.standard_normal(L // 2 + 3).astype(np.float32)),
+            np.float32(rng.integers(0, 2, 2000))]
+    idx, sc, lens = _topk_rows(rows, 2048)
+    assert np.array_equal(idx, oracle.topk(sc.astype(np.float64), lens, 2048))
+    assert list(idx[0]) == list(range(2048))
+
+
 def test_topk_streaming_rows_unaligned():
     """Rows above 16384 positions stream from memory; an odd row stride leaves
     all but the first row unaligned (positions load one at a time) and the
