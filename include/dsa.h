@@ -245,7 +245,12 @@ dsa_status dsa_sparse_mla_attn(const dsa_batch *batch, const dsa_mla_in *in, con
                                dsa_stream_t stream);
 
 /* The whole decode chain: indexer scores -> Top-K -> sparse MLA, enqueued
- * back to back on `stream` with intermediates in the workspace.
+ * back to back on `stream` with intermediates in the workspace. The three
+ * kernels are chained with programmatic dependent launch: the first one may
+ * be scheduled while the stream's previous kernel finishes, but waits for it
+ * before reading any input, so inputs written by earlier work on the stream
+ * (including a kernel that itself allows programmatic dependents) are seen
+ * complete.
  * idx_out: if non-NULL, int32 [T, k] receives the selected indices.
  * stage_events: NULL, or 4 caller-created events recorded before the indexer,
  *   before the Top-K, before the attention and after the attention (timing).

@@ -878,10 +878,13 @@ dsa_status dsa_fused_decode(const dsa_batch* batch, const dsa_indexer_in* idx_in
     const cudaError_t e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), st);
     return e == cudaSuccess ? DSA_OK : fail(DSA_ERR_CUDA, "cudaEventRecord: %s", cudaGetErrorString(e));
   };
-  // Programmatic dependent launch on every edge: each kernel's prologue
-  // overlaps the tail of the previous one (for the indexer: the previous
-  // call's attention) and waits on the device for what it consumes. Not used
-  // when stage events sit between the kernels.
+  // Programmatic dependent launch on every edge: each kernel is scheduled
+  // while the previous one finishes and waits on the device for what it
+  // consumes. The indexer waits before it reads anything (whatever ran
+  // before the call may have written its inputs) and only then lets the
+  // Top-K be scheduled, so the Top-K and the attention, which read the
+  // batch description and the queries before their own waits, see complete
+  // inputs. Not used when stage events sit between the kernels.
   const bool pdl = stage_events == nullptr;
   if ((s = rec(0)) != DSA_OK) return s;
   if ((s = launch_indexer(batch, idx_in, scores, batch->max_seq_len, st, pdl,

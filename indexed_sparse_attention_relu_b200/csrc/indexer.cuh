@@ -119,6 +119,11 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
 
   const int warp = warp_id();
   const int lane = lane_id();
+  // Under programmatic dependent launch this grid may start before the
+  // previous kernel of the stream has finished, and that kernel may have
+  // written any input, so nothing is read before the wait. Only then may the
+  // Top-K be scheduled: it reads the batch description before its own wait.
+  pdl_wait_prior();
   pdl_launch_dependents();  // the Top-K may be scheduled; it waits for these scores
   if (threadIdx.x == 0) prefetch_tensormap(&kmap);
 
@@ -215,10 +220,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
   const int b = misc[0];
   const int tile_begin = misc[3];
   const int tile_end = misc[4];
-  if (b < 0 || tile_begin >= tile_end) {  // uniform across the CTA
-    pdl_wait_prior();
-    return;
-  }
+  if (b < 0 || tile_begin >= tile_end) return;  // uniform across the CTA
   const int t0 = misc[1];
   const int nt = misc[2];
   const int nk = misc[12];  // causal candidates of the group's last token
@@ -543,12 +545,6 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
   canary_check(smem, C::SMEM_BYTES);
-  // Under programmatic dependent launch this grid may start while the
-  // previous kernel of the stream (the attention of the previous call) still
-  // runs. It reads nothing that kernel writes, but it must not complete
-  // before it: the next kernel (Top-K) waits only for this grid and then
-  // rewrites the indices the attention reads.
-  pdl_wait_prior();
 }
 
 }  // namespace dsa

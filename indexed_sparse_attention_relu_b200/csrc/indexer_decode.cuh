@@ -133,6 +133,12 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, KF>::THREADS, 1)
   float* w_s = reinterpret_cast<float*>(smem + C::OFF_W);
   const int warp = warp_id();
   const int lane = lane_id();
+  // Under programmatic dependent launch this grid may start before the
+  // previous kernel of the stream has finished, and that kernel may have
+  // written any input (queries, keys, weights, the batch description), so
+  // nothing is read before the wait. Only then may the Top-K be scheduled: it
+  // reads the batch description before its own wait.
+  pdl_wait_prior();
   pdl_launch_dependents();  // the Top-K may be scheduled; it waits for these scores
 
   if (warp == 0) {
@@ -542,11 +548,6 @@ __global__ void __launch_bounds__(IdxDecCfg<HI, DIN, KF>::THREADS, 1)
     tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
   canary_check(smem, C::SMEM_BYTES);
-  // Under programmatic dependent launch this grid may start while the
-  // previous kernel of the stream still runs. It reads nothing that kernel
-  // writes, but it must not complete before it: the next kernel (Top-K)
-  // waits only for this grid and then rewrites what that kernel reads.
-  pdl_wait_prior();
 }
 
 }  // namespace dsa

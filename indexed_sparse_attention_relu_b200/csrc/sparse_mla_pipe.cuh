@@ -650,7 +650,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       __syncwarp();
     }
 
-    // ------------------------------------------------------------ epilogue (warps 0-19)
+    // ------------------------------------------------------------ epilogue (warps 0-11)
     // O is final once the drain commit has landed. Warps w, w + 4, ... read
     // the same 32 TMEM lanes (32 (w % 4) ...) and split the 32 chunks of 16
     // columns between them.
