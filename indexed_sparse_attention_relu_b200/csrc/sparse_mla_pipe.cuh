@@ -285,8 +285,9 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
       for (int j = 0; j < n_tiles; ++j) {
         const int i0 = (j * C::TK + lane < nk) ? sidx[j * C::TK + lane] : -1;
         const int i1 = (j * C::TK + 32 + lane < nk) ? sidx[j * C::TK + 32 + lane] : -1;
-        const unsigned v0 = __ballot_sync(0xffffffffu, i0 >= 0 && i0 < len);
-        const unsigned v1 = __ballot_sync(0xffffffffu, i1 >= 0 && i1 < len);
+        // staged entries: positions (contiguous) or pool rows with -1 for masked keys (paged)
+        const unsigned v0 = __ballot_sync(0xffffffffu, i0 >= 0 && (PAGED || i0 < len));
+        const unsigned v1 = __ballot_sync(0xffffffffu, i1 >= 0 && (PAGED || i1 < len));
         float v[64];
         if (ok) ok = mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, abort_flag);
         if (ok) {
@@ -409,6 +410,22 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
             const int i = base + u * GT + gl;
             v[u] = i < nk ? ld_dep(idx_row + k_begin + i) : -1;
           }
+          if constexpr (PAGED) {
+            // paged caches: each selected row's pool position, looked up once
+            // here rather than before every gather; -1 marks a masked key (-1,
+            // or a position outside the sequence, which is reported)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int i = base + u * GT + gl;
+              const int s = v[u];
+              if (s >= 0 && s < len) {
+                v[u] = p.cm.row_checked(b, s);
+              } else {
+                if (i < nk && s != -1) set_device_status(DSA_ERR_DEVICE_INDEX);
+                v[u] = -1;
+              }
+            }
+          }
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int i = base + u * GT + gl;
@@ -438,15 +455,16 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
         if (!reinterpret_cast<volatile int*>(misc)[4 + (j & 1)]) break;
         if (active) {
           int y[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const bool v = cur[i] >= 0 && cur[i] < len;
-            if (a == 0 && cur[i] != -1 && !v) set_device_status(DSA_ERR_DEVICE_INDEX);
-            y[i] = row0 + (v ? cur[i] : 0);
-          }
           if constexpr (PAGED) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) y[i] = (cur[i] >= 0 && cur[i] < len) ? p.cm.row_checked(b, cur[i]) : 0;
+            for (int i = 0; i < 4; ++i) y[i] = cur[i] >= 0 ? cur[i] : 0;  // staged pool rows (masked: row 0)
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const bool v = cur[i] >= 0 && cur[i] < len;
+              if (a == 0 && cur[i] != -1 && !v) set_device_status(DSA_ERR_DEVICE_INDEX);
+              y[i] = row0 + (v ? cur[i] : 0);
+            }
           }
           tma_gather4(smem_u32(smem + C::A_OFF_K + sl * C::K_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0], y[1],
                       y[2], y[3], &kv_full[sl]);
@@ -565,11 +583,23 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           y[i] = (active && tile < n_tiles && k < k_end) ? ld_dep(idx_row + k) : -1;
         }
       };
+      // paged caches: the pool rows of the next tile are looked up one tile
+      // ahead (from positions loaded three tiles before), so the block-table
+      // load is not waited on right before a gather
+      auto pool_rows = [&](const int (&s)[4], int (&y)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          bool rok;
+          y[i] = (s[i] >= 0 && s[i] < len) ? p.cm.row(b, s[i], rok) : 0;
+        }
+      };
       int r0[4], r1[4], r2[4], r3[4];
       load_rows(0, r0);
       load_rows(1, r1);
       load_rows(2, r2);
       load_rows(3, r3);
+      int pr[4] = {0, 0, 0, 0};  // pool rows of the tile issued next (paged)
+      if constexpr (PAGED) pool_rows(r0, pr);
       int issued = 0;
       bool stop = false;
       for (int j0 = 0; j0 < n_tiles && !stop; j0 += 4) {
@@ -578,6 +608,7 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           const int j = j0 + u;
           if (j >= n_tiles || stop) break;
           int (&cur)[4] = u == 0 ? r0 : u == 1 ? r1 : u == 2 ? r2 : r3;
+          const int (&nxt)[4] = u == 0 ? r1 : u == 1 ? r2 : u == 2 ? r3 : r0;  // tile j + 1's positions
           const int sl = j % C::NVS;
           if (leader) {
             const bool ok = mbar_wait(&v_empty[sl], ((j / C::NVS) & 1) ^ 1u, abort_flag);
@@ -591,19 +622,18 @@ __global__ void __launch_bounds__(PipeCfg::THREADS, 1)
           }
           if (active) {
             int y[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) y[i] = row0 + ((cur[i] >= 0 && cur[i] < len) ? cur[i] : 0);
             if constexpr (PAGED) {
 #pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                bool rok;
-                y[i] = (cur[i] >= 0 && cur[i] < len) ? p.cm.row(b, cur[i], rok) : 0;
-              }
+              for (int i = 0; i < 4; ++i) y[i] = pr[i];
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) y[i] = row0 + ((cur[i] >= 0 && cur[i] < len) ? cur[i] : 0);
             }
             tma_gather4(smem_u32(smem + C::B_OFF_V + sl * C::V_BYTES + a * C::ATOM + g * 512), &kvmap, a * 64, y[0],
                         y[1], y[2], y[3], &v_full[sl]);
           }
           ++issued;
+          if constexpr (PAGED) pool_rows(nxt, pr);
           load_rows(j + 4, cur);
         }
       }
