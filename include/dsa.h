@@ -365,6 +365,15 @@ dsa_status dsa_read_device_status(dsa_stream_t stream, int32_t *code_out);
 dsa_status dsa_debug_set_wait_limit(uint64_t limit_ns);
 dsa_status dsa_debug_withhold_signal(int32_t on);
 
+/* Test hook for the ordering of the chained calls: enqueues on `stream` a
+ * kernel that lets programmatically dependent launches start at once, then
+ * waits delay_ns (at most 1 s) and only then copies `bytes` from src to dst
+ * (device memory; both addresses and bytes multiples of 16). A call enqueued
+ * next on the stream must still see dst's new contents.
+ * DSA_ERR_INVALID_ARGUMENT for NULL, misaligned or too long a delay. */
+dsa_status dsa_debug_delayed_copy(void *dst, const void *src, size_t bytes, uint64_t delay_ns,
+                                  dsa_stream_t stream);
+
 /* Text for a status code (static storage). */
 const char *dsa_status_string(dsa_status s);
 

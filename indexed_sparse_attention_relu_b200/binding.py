@@ -49,7 +49,7 @@ EXPORTED = (
     "dsa_quantize_mxfp8",
     "dsa_workspace_size",
     "dsa_read_device_status", "dsa_status_string", "dsa_last_error", "dsa_version",
-    "dsa_debug_set_wait_limit", "dsa_debug_withhold_signal",
+    "dsa_debug_set_wait_limit", "dsa_debug_withhold_signal", "dsa_debug_delayed_copy",
 )
 
 
@@ -108,6 +108,7 @@ def load() -> ctypes.CDLL:
             "dsa_version": (c_char_p, []),
             "dsa_debug_set_wait_limit": (c_int, [ctypes.c_uint64]),
             "dsa_debug_withhold_signal": (c_int, [c_int32]),
+            "dsa_debug_delayed_copy": (c_int, [P, P, c_size_t, ctypes.c_uint64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -282,3 +283,11 @@ def dsa_debug_set_wait_limit(limit_ns: int) -> None:
 def dsa_debug_withhold_signal(on: bool) -> None:
     """Test hook: the 128-head attention withholds its first P-ready signal."""
     _check(load().dsa_debug_withhold_signal(1 if on else 0))
+
+
+def dsa_debug_delayed_copy(dst: torch.Tensor, src: torch.Tensor, delay_ns: int, stream=None) -> None:
+    """Test hook: a kernel that lets dependent launches start at once, sleeps
+    delay_ns, then copies src into dst (same byte size)."""
+    nbytes = dst.numel() * dst.element_size()
+    assert src.numel() * src.element_size() == nbytes
+    _check(load().dsa_debug_delayed_copy(_ptr(dst), _ptr(src), nbytes, int(delay_ns), _stream(stream)))

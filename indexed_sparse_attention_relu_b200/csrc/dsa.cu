@@ -762,6 +762,19 @@ dsa_status launch_mla(const dsa_batch* bt, const dsa_mla_in* in, const int32_t* 
   return launch_mla_t<80, 64>(bt, in, idx, k, out, lse, ws, ws_bytes, st, pl, pdl);
 }
 
+// Test hook: a kernel that lets programmatic dependents start at once, then
+// waits delay_ns of wall time (a bounded sleep loop) and only then copies src
+// to dst, so a dependent that read dst before its own wait would see the old
+// contents.
+__global__ void debug_delayed_copy_kernel(uint4* dst, const uint4* src, int64_t n16, uint64_t delay_ns) {
+  pdl_launch_dependents();
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < delay_ns) __nanosleep(2000);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -1008,6 +1021,17 @@ dsa_status dsa_debug_set_wait_limit(uint64_t limit_ns) {
   const cudaError_t e = cudaMemcpyToSymbol(dsa::g_wait_limit_ns, &v, sizeof(v));
   if (e != cudaSuccess) return fail(DSA_ERR_CUDA, "setting the wait limit: %s", cudaGetErrorString(e));
   return DSA_OK;
+}
+
+dsa_status dsa_debug_delayed_copy(void* dst, const void* src, size_t bytes, uint64_t delay_ns, dsa_stream_t stream) {
+  if (!dst || !src) return fail(DSA_ERR_INVALID_ARGUMENT, "dst and src must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | bytes) & 15u)
+    return fail(DSA_ERR_INVALID_ARGUMENT, "dst, src and bytes must be multiples of 16");
+  if (delay_ns > 1000000000ull) return fail(DSA_ERR_INVALID_ARGUMENT, "delay_ns above 1 s");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  debug_delayed_copy_kernel<<<64, 256, 0, st>>>(static_cast<uint4*>(dst), static_cast<const uint4*>(src),
+                                                 static_cast<int64_t>(bytes / 16), delay_ns);
+  return check_launch("debug_delayed_copy");
 }
 
 dsa_status dsa_debug_withhold_signal(int32_t on) {
