@@ -25,8 +25,8 @@
 // copied into the stage with the codes when their rows are 16-byte aligned.
 //
 // Roles: warp 0 = TMA producer, warp 1 = MMA issuer (+ TMEM owner), then the
-// epilogue warps (four; eight for multi-token groups, two per TMEM
-// sub-partition splitting the tokens), then four FP8 converters (FP8 only).
+// epilogue warps (four; for groups of 64-head tokens up to four per TMEM
+// sub-partition, splitting the tokens), then four FP8 converters (FP8 only).
 #pragma once
 #include "dsa_common.cuh"
 #include "quant.cuh"
@@ -68,9 +68,12 @@ struct IndexerCfg {
   static constexpr int NACC = 2;                           // TMEM accumulator buffers
   static constexpr int TMEM_COLS = (NACC * N <= 32) ? 32 : (NACC * N <= 64) ? 64 : (NACC * N <= 128) ? 128
                                    : (NACC * N <= 256) ? 256 : 512;
-  // epilogue warps: two per TMEM sub-partition for multi-token groups (each
-  // takes half of the tokens), one otherwise
-  static constexpr int EPI_WARPS = (G > 1 && HI % 64 == 0 && G % 2 == 0) ? 8 : 4;
+  // epilogue warps: EPI_PARTS per TMEM sub-partition, each taking G / EPI_PARTS
+  // of the group's tokens (64-head tokens: four parts for four-token groups of
+  // BF16 keys; with 8-bit keys the converter warps leave registers for two)
+  static constexpr int EPI_PARTS =
+      (G > 1 && HI % 64 == 0) ? ((G % 4 == 0 && KF == 0) ? 4 : G % 2 == 0 ? 2 : 1) : 1;
+  static constexpr int EPI_WARPS = 4 * EPI_PARTS;
   static constexpr int NUM_WARPS = 2 + EPI_WARPS + (FP8 ? 4 : 0);
   static constexpr int THREADS = NUM_WARPS * 32;
   // shared memory carve-up (offsets from a 1024-aligned base)
@@ -370,7 +373,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
   } else if (warp >= 2 && warp < 2 + C::EPI_WARPS) {
     // ------------------------------------------------------------ epilogue
     const int sub = warp & 3;                 // TMEM sub-partition this warp may access
-    const int part = (warp - 2) / 4;          // token half (eight epilogue warps) or 0
+    const int part = (warp - 2) / 4;          // this warp's share of the group's tokens
     const int r = sub * 32 + lane;            // key row inside the tile
     const uint32_t lane_addr = static_cast<uint32_t>(sub * 32) << 16;
     int nv[G];
@@ -400,9 +403,9 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
         }
       } else if constexpr (HI % 64 == 0) {
         // wide tiles, 64 heads per token: one token's 64 columns per TMEM
-        // round trip (four loads in flight, one wait); with eight epilogue
-        // warps each takes the columns of its half of the tokens
-        constexpr int COLS = C::EPI_WARPS == 8 ? C::N / 2 : C::N;
+        // round trip (four loads in flight, one wait); each warp takes the
+        // columns of its share of the tokens
+        constexpr int COLS = C::N / C::EPI_PARTS;
 #pragma unroll 1
         for (int c = part * COLS; c < (part + 1) * COLS; c += 64) {
           float v[4][16];
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
         }
       }
       if (s < p.ld) {
-        constexpr int GPART = C::EPI_WARPS == 8 ? G / 2 : G;  // tokens this warp scores
+        constexpr int GPART = G / C::EPI_PARTS;  // tokens this warp scores
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           if (g < nt && g / GPART == part) {
