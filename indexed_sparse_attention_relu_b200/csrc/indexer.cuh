@@ -74,7 +74,8 @@ struct IndexerCfg {
   static constexpr int EPI_PARTS =
       (G > 1 && HI % 64 == 0) ? ((G % 4 == 0 && KF == 0) ? 4 : G % 2 == 0 ? 2 : 1) : 1;
   static constexpr int EPI_WARPS = 4 * EPI_PARTS;
-  static constexpr int NUM_WARPS = 2 + EPI_WARPS + (FP8 ? 4 : 0);
+  static constexpr int CONV_WARPS = FP8 ? 4 : 0;          // 8-bit -> bf16 converters
+  static constexpr int NUM_WARPS = 2 + EPI_WARPS + CONV_WARPS;
   static constexpr int THREADS = NUM_WARPS * 32;
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
@@ -205,14 +206,14 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
       misc[6] = 0;
       for (int i = 0; i < C::ST; ++i) {
         mbar_init(&full[i], 1);
-        mbar_init(&empty[i], FP8 ? 4 : 1);
+        mbar_init(&empty[i], FP8 ? C::CONV_WARPS : 1);
       }
       for (int i = 0; i < C::NACC; ++i) {
         mbar_init(&acc_full[i], 1);
         mbar_init(&acc_empty[i], C::EPI_WARPS);
       }
       for (int i = 0; i < C::CS; ++i) {
-        mbar_init(&conv_full[i], 4);
+        mbar_init(&conv_full[i], C::CONV_WARPS);
         mbar_init(&conv_empty[i], 1);
       }
       mbar_init(drain, 1);
@@ -466,7 +467,8 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
     }
   } else if constexpr (FP8) {
     // ------------------------------------------------------------ FP8 -> bf16 converters
-    const int ct = threadIdx.x - (2 + C::EPI_WARPS) * 32;  // 0..127
+    constexpr int CT = 32 * C::CONV_WARPS;                 // converter threads
+    const int ct = threadIdx.x - (2 + C::EPI_WARPS) * 32;  // 0 .. CT - 1
     constexpr int CPR = DIN / 16;         // 16-byte input chunks per key row
     for (int it = 0; it < n_tiles; ++it) {
       const int st = it % C::ST;
@@ -477,12 +479,13 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
       uint8_t* dst = smem + C::OFF_CONV + cs * C::TILE_BYTES;
       const int s0 = (tile_begin + it) * 128;  // first key position of the tile
       // all of the thread's chunks (and MXFP8 scale bytes) are loaded first
-      constexpr int PER = (128 * CPR + 127) / 128;
+      static_assert((128 * CPR) % CT == 0, "whole chunks per converter thread");
+      constexpr int PER = 128 * CPR / CT;
       uint4 raws[PER];
       int bytes[PER];
 #pragma unroll
       for (int u = 0; u < PER; ++u) {
-        const int i = ct + u * 128;
+        const int i = ct + u * CT;
         const int row = i / CPR;
         const int c = i % CPR;
         raws[u] = *reinterpret_cast<const uint4*>(src + row * DIN + c * 16);
@@ -500,7 +503,7 @@ __global__ void __launch_bounds__(IndexerCfg<HI, DIN, G, KF>::THREADS, IndexerCf
       }
 #pragma unroll
       for (int u = 0; u < PER; ++u) {
-        const int i = ct + u * 128;
+        const int i = ct + u * CT;
         const int row = i / CPR;
         const int c = i % CPR;
         const uint32_t words[4] = {raws[u].x, raws[u].y, raws[u].z, raws[u].w};
