@@ -20,7 +20,7 @@
 // tcgen05.mma with M = 128 keys, N = heads, K = d_I into two TMEM
 // accumulators. Epilogue warps read one key row per thread, apply ReLU,
 // the weights, the key's scale (FP8) and the causal / length mask and store
-// the scores. FP8 codes are widened to bf16 by four converter warps (exact:
+// the scores. 8-bit codes are widened to bf16 by converter warps (exact:
 // every E4M3 value is a bf16). Key formats (KF): BF16; FP8 with one fp32 scale
 // per key, applied after the head sum; MXFP8 with one power-of-two (E8M0)
 // scale per 32 elements, applied by the converters while widening (still
