@@ -12,7 +12,7 @@
 // Design (swapped AB): one tcgen05.mma tile is M = 128 keys x N = G tokens x
 // H_I heads x K = d_I, so the large operand (the key cache, streamed from HBM
 // by TMA) is A and the small one (the group's queries, resident in shared
-// memory) is B. The fp32 accumulator lives in TMEM (two buffers); four
+// memory) is B. The fp32 accumulator lives in TMEM (two buffers); the
 // epilogue warps read one key row per thread with tcgen05.ld, apply ReLU, the
 // head weights, the FP8 scale and the causal / length mask, and store the
 // scores coalesced. FP8 keys are TMA-loaded as bytes and widened to bf16 in
