@@ -233,3 +233,15 @@ def test_header_page_size_rule_matches_validation(lib):
         want = B.DSA_OK if ps % mult == 0 else B.DSA_ERR_UNSUPPORTED_SHAPE
         b = _batch(num_q=0, block_table=FAKE, page_size=ps, num_pages=4)
         assert _scores(lib, b, _idx_in()) == want, ps
+
+
+def test_delayed_copy_hook_validation(lib):
+    """The ordering test hook rejects what it cannot copy before it launches
+    anything: NULL pointers, addresses or sizes that are not multiples of 16
+    bytes, and delays above one second."""
+    h = lib.dsa_debug_delayed_copy
+    assert h(None, FAKE, 64, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert h(FAKE, None, 64, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert h(MIS, FAKE, 64, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert h(FAKE, FAKE, 60, 0, None) == B.DSA_ERR_INVALID_ARGUMENT
+    assert h(FAKE, FAKE, 64, 1_000_000_001, None) == B.DSA_ERR_INVALID_ARGUMENT
